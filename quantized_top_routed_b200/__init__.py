@@ -2,13 +2,6 @@
 
 The compute lives in ``libqmoe.so`` (CUDA kernels behind a C ABI declared in
 ``include/qmoe.h``).  ``quantized_top_routed_b200.qmoe`` is the thin ctypes
-binding with the same call names; ``synth`` makes seeded inputs.
+binding with the same call names; ``synth`` makes seeded inputs.  Import the
+submodules directly.
 """
-__all__ = ["synth", "qmoe"]
-
-
-def __getattr__(name):
-    if name == "qmoe":
-        from . import qmoe as _q
-        return _q
-    raise AttributeError(name)

@@ -1,0 +1,251 @@
+// Internal declarations and sm_100a PTX wrappers for libqmoe.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/qmoe.h"
+
+namespace qmoe {
+
+constexpr int kMaxE = 256;        // routed experts
+constexpr int kMaxK = 16;         // experts per token
+constexpr int kMaxShared = 8;     // shared experts
+constexpr int kBK = 128;          // K elements per pipeline stage of the grouped GEMMs
+constexpr int kTileM = 128;       // weight rows per GEMM tile (MMA M)
+
+// Error bits written to the handle's device error word.
+constexpr int kErrTimeout = 1;
+
+// One expert's weights after repacking (device pointers, owned by the handle).
+// mat 0 = gate/up (W13, K = d), mat 1 = down (W2, K = I).
+struct ExpertDev {
+  const uint8_t* w[2];     // tile blobs: [m_block][k_stage] of stage_bytes(fmt)
+  const float* spc[2];     // per-channel scales in tile-row order (INT8 / FP8), else nullptr
+  int32_t fmt;
+  int32_t pad;
+};
+
+// Bytes of one repacked (128 rows x 128 K) tile.  INT4 tiles carry their
+// 128 bf16 group scales after the codes.
+__host__ __device__ inline int stage_bytes(int fmt) {
+  return fmt == QMOE_W_INT4_G128 ? (128 * 64 + 256) : (128 * 128);
+}
+
+// Arguments of the grouped GEMM kernels.
+struct GemmArgs {
+  const ExpertDev* experts;   // [n_seg]
+  int mat;                    // 0: gate/up (gated SwiGLU epilogue), 1: down
+  const uint16_t* act;        // B operand rows (bf16): x [T][d] (gathered) or H [P][I]
+  int act_ld;                 // elements per act row
+  const int32_t* gather;      // row -> act row (sorted_token) or nullptr for identity
+  const int32_t* seg_off;     // [n_seg] first permuted row of each segment
+  const int32_t* seg_cnt;     // [n_seg] rows in each segment
+  const int32_t* tile_off;    // [n_seg + 1] prefix sum of tiles per segment
+  int n_seg;
+  int K;                      // reduction length (d or I)
+  int MB;                     // 128-row weight blocks per expert matrix
+  uint16_t* out;              // H [P][I] or Y [P][d]
+  int out_ld;
+  int* err;                   // device error word
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar_addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity.  Gives up (returns
+// false) when *abort is raised by another role or after ~2^31 SM cycles
+// (about a second), in which case it raises *abort itself.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  const uint32_t addr = smem_u32(bar);
+  if (mbar_try_wait(addr, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(addr, parity)) return true;
+    if ((i & 255u) == 0) {
+      if (*abort) return false;
+      if (clock64() - t0 > (1ll << 31)) {
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// Same, ignoring the abort flag (used while draining on the way out).
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  const uint32_t addr = smem_u32(bar);
+  const long long t0 = clock64();
+  while (!mbar_try_wait(addr, parity)) {
+    if (clock64() - t0 > (1ll << 30)) return false;
+  }
+  return true;
+}
+
+// 1-D bulk copy global -> shared, completion counted on an mbarrier (bytes).
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// 16-byte cp.async with zero fill of the bytes beyond src_bytes (0 or 16).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// --- tcgen05 ---------------------------------------------------------------
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Whole warp: allocate ncols TMEM columns, address written to *slot.
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16 (bf16 inputs, fp32 accumulate).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on an mbarrier once all previously issued tcgen05 ops of this thread complete.
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 32 lanes x 16 consecutive 32-bit columns -> 16 registers per thread.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+// 16 registers per thread -> 32 lanes x 16 consecutive columns.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+// Instruction descriptor, kind::f16: bf16 A and B (both K-major), fp32 D, M = 128.
+__host__ __device__ constexpr uint32_t idesc_bf16_m128(int n) {
+  return (1u << 4)                          // D format: f32
+         | (1u << 7)                        // A format: bf16
+         | (1u << 10)                       // B format: bf16
+         | ((uint32_t)(n >> 3) << 17)       // N / 8
+         | ((uint32_t)(128 >> 4) << 24);    // M / 16
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (the stage buffers are 1024-byte aligned).
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu)   // start address
+         | ((uint64_t)1 << 16)                // leading byte offset (unused with swizzle)
+         | ((uint64_t)(1024 >> 4) << 32)      // stride byte offset
+         | ((uint64_t)1 << 46)                // descriptor version (sm_100)
+         | ((uint64_t)2 << 61);               // SWIZZLE_128B
+}
+
+// ---------------------------------------------------------------------------
+// host-side launchers (implemented in the .cu files)
+// ---------------------------------------------------------------------------
+cudaError_t launch_router_logits(const uint16_t* x, const float* Wr, int T, int d, int E, int split,
+                                 float* zpart, cudaStream_t s);
+cudaError_t launch_router_topk(const float* zpart, int split, const float* bias, int T, int E, int k,
+                               int32_t* idx, float* gate, cudaStream_t s);
+int router_split(int T, int d, int E, int num_sms);
+
+cudaError_t launch_schedule(const int32_t* idx, int T, int k, int E, int S, int bn3, int mb3, int bn4, int mb4,
+                            int32_t* counts, int32_t* offsets, int32_t* sorted_token, int32_t* inv_pos,
+                            int32_t* seg_off, int32_t* seg_cnt, int32_t* tile3_off, int32_t* tile4_off,
+                            int32_t* scratch, cudaStream_t s);
+size_t schedule_scratch_ints(int max_tokens, int E);
+
+cudaError_t launch_grouped_gemm(const GemmArgs& a, int bn, int num_sms, cudaStream_t s);
+bool gemm_bn_supported(int bn);
+
+cudaError_t launch_combine(const uint16_t* Y, const float* gate, const int32_t* inv_pos, int T, int k, int S,
+                           int d, uint16_t* out, cudaStream_t s);
+
+cudaError_t launch_repack(int fmt, int mat, const void* w, const void* scale, int rows, int K, int I,
+                          uint8_t* dst, float* dst_spc, cudaStream_t s);
+
+}  // namespace qmoe

@@ -1,0 +1,168 @@
+// Stage 2: expert-centric schedule.  Every (token, slot) decision is a task;
+// tasks are grouped by expert id and sorted by token id inside each group,
+// so each expert's rows are contiguous for the grouped GEMMs.  ("OmniMoE: An
+// Efficient MoE by Orchestrating Atomic Experts at Scale", section 2.2,
+// Expert-Centric Scheduling: task collection, grouping and sorting.)
+//
+// One CTA of 1024 threads, deterministic (no atomics decide any position):
+//   phase 1: each warp takes chunks of 32 tokens; for every expert a warp
+//            ballot gives the chunk's count and each task's rank among the
+//            chunk's earlier tokens;
+//   phase 2: per expert, an exclusive scan of the chunk counts (the chunk's
+//            base inside the expert's segment), the expert totals and the
+//            exclusive scan over experts (offsets);
+//   phase 3: pos(t, j) = offsets[e] + base[chunk][e] + rank; scatter.
+// It also writes the segment table (routed experts, then one identity
+// segment of T rows per shared expert) and, per grouped GEMM, the prefix sum
+// of its tiles per segment, so the GEMMs never need the counts on the host.
+#include "qmoe_internal.cuh"
+
+namespace qmoe {
+namespace {
+
+constexpr int kThreads = 1024;
+
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, v, off);
+    if (lane >= off) v += o;
+  }
+  return v;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    schedule_kernel(const int32_t* __restrict__ idx, int T, int k, int E, int S, int bn3, int mb3, int bn4,
+                    int mb4, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                    int32_t* __restrict__ sorted_token, int32_t* __restrict__ inv_pos,
+                    int32_t* __restrict__ seg_off, int32_t* __restrict__ seg_cnt, int32_t* __restrict__ tile3_off,
+                    int32_t* __restrict__ tile4_off, int32_t* __restrict__ hist) {
+  __shared__ uint32_t bal[32][kMaxE];
+  __shared__ int32_t s_cnt[kMaxE + kMaxShared];
+  __shared__ int32_t s_off[kMaxE + 1];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int C = (T + 31) / 32;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+
+  // ---- phase 1: per-chunk counts and in-chunk ranks ------------------------
+  for (int c = warp; c < C; c += 32) {
+    const int t = c * 32 + lane;
+    const bool valid = t < T;
+    for (int w0 = 0; w0 < E; w0 += 32) {
+      uint32_t m = 0;
+      if (valid)
+        for (int j = 0; j < k; ++j) {
+          const int e = idx[(size_t)t * k + j] - w0;
+          if (e >= 0 && e < 32) m |= 1u << e;
+        }
+      uint32_t mine = 0;
+#pragma unroll 8
+      for (int b = 0; b < 32; ++b) {
+        const uint32_t v = __ballot_sync(0xffffffffu, (m >> b) & 1u);
+        if (lane == b) mine = v;
+      }
+      if (w0 + lane < E) {
+        bal[warp][w0 + lane] = mine;
+        hist[(size_t)c * E + w0 + lane] = __popc(mine);
+      }
+    }
+    __syncwarp();
+    if (valid)
+      for (int j = 0; j < k; ++j) {
+        const int e = idx[(size_t)t * k + j];
+        inv_pos[(size_t)t * k + j] = __popc(bal[warp][e] & lt_mask);  // rank for now
+      }
+    __syncwarp();
+  }
+  __syncthreads();
+
+  // ---- phase 2: chunk bases per expert, expert totals, offsets -------------
+  for (int e = warp; e < E; e += 32) {
+    const int per = (C + 31) / 32;
+    const int c0 = min(C, lane * per), c1 = min(C, c0 + per);
+    int sum = 0;
+    for (int c = c0; c < c1; ++c) sum += hist[(size_t)c * E + e];
+    const int incl = warp_incl_scan(sum, lane);
+    int run = incl - sum;
+    for (int c = c0; c < c1; ++c) {
+      const int h = hist[(size_t)c * E + e];
+      hist[(size_t)c * E + e] = run;
+      run += h;
+    }
+    if (lane == 31) s_cnt[e] = incl;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int running = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int v = (e0 + lane < E) ? s_cnt[e0 + lane] : 0;
+      const int incl = warp_incl_scan(v, lane);
+      if (e0 + lane < E) s_off[e0 + lane] = running + incl - v;
+      running += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) s_off[E] = running;
+  }
+  __syncthreads();
+
+  // ---- phase 3: scatter -----------------------------------------------------
+  const int P = T * k;
+  for (int p = tid; p < P; p += kThreads) {
+    const int t = p / k;
+    const int e = idx[p];
+    const int pos = s_off[e] + hist[(size_t)(t >> 5) * E + e] + inv_pos[p];
+    sorted_token[pos] = t;
+    inv_pos[p] = pos;
+  }
+  for (int e = tid; e < E; e += kThreads) counts[e] = s_cnt[e];
+  for (int e = tid; e <= E; e += kThreads) offsets[e] = s_off[e];
+  for (int p = tid; p < S * T; p += kThreads) sorted_token[P + p] = p % T;
+
+  // ---- segment and tile tables for the grouped GEMMs ------------------------
+  if (seg_off == nullptr) return;
+  const int n_seg = E + S;
+  if (warp == 0) {
+    int run3 = 0, run4 = 0;
+    for (int e0 = 0; e0 < n_seg; e0 += 32) {
+      const int e = e0 + lane;
+      int cnt = 0, off = 0;
+      if (e < E) {
+        cnt = s_cnt[e];
+        off = s_off[e];
+      } else if (e < n_seg) {
+        cnt = T;
+        off = P + (e - E) * T;
+      }
+      const int t3 = ((cnt + bn3 - 1) / bn3) * mb3;
+      const int t4 = ((cnt + bn4 - 1) / bn4) * mb4;
+      const int i3 = warp_incl_scan(t3, lane);
+      const int i4 = warp_incl_scan(t4, lane);
+      if (e < n_seg) {
+        seg_off[e] = off;
+        seg_cnt[e] = cnt;
+        tile3_off[e] = run3 + i3 - t3;
+        tile4_off[e] = run4 + i4 - t4;
+      }
+      run3 += __shfl_sync(0xffffffffu, i3, 31);
+      run4 += __shfl_sync(0xffffffffu, i4, 31);
+    }
+    if (lane == 0) {
+      tile3_off[n_seg] = run3;
+      tile4_off[n_seg] = run4;
+    }
+  }
+}
+
+}  // namespace
+
+size_t schedule_scratch_ints(int max_tokens, int E) { return (size_t)((max_tokens + 31) / 32) * E; }
+
+cudaError_t launch_schedule(const int32_t* idx, int T, int k, int E, int S, int bn3, int mb3, int bn4, int mb4,
+                            int32_t* counts, int32_t* offsets, int32_t* sorted_token, int32_t* inv_pos,
+                            int32_t* seg_off, int32_t* seg_cnt, int32_t* tile3_off, int32_t* tile4_off,
+                            int32_t* scratch, cudaStream_t s) {
+  schedule_kernel<<<1, kThreads, 0, s>>>(idx, T, k, E, S, bn3, mb3, bn4, mb4, counts, offsets, sorted_token, inv_pos,
+                                         seg_off, seg_cnt, tile3_off, tile4_off, scratch);
+  return cudaGetLastError();
+}
+
+}  // namespace qmoe

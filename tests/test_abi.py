@@ -1,0 +1,88 @@
+"""The C-ABI library builds, loads and exports what include/qmoe.h declares (CPU only).
+
+Only calls that fail argument validation before touching CUDA are made here.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from quantized_top_routed_b200 import qmoe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    with open(os.path.join(ROOT, "include", "qmoe.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qmoe_[a-z_]+)\s*\(", text)))
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = qmoe.load()
+    names = declared_functions()
+    assert len(names) >= 8
+    for name in names:
+        assert hasattr(lib, name), f"{name} declared in qmoe.h but not exported"
+    assert set(names) == set(qmoe.EXPORTS)
+
+
+def test_symbols_are_c_linkage():
+    out = os.popen(f"nm -D --defined-only {qmoe.library_path()}").read()
+    for name in declared_functions():
+        assert re.search(rf"\sT {name}$", out, flags=re.M), name
+
+
+def test_destroy_null_is_ok_and_last_error_is_a_string():
+    qmoe.qmoe_destroy(None)
+    assert isinstance(qmoe.qmoe_last_error(), str)
+
+
+def _create_raw(cfg, router_w=1, experts_n=1, fmt=1, ptrs=(16, 16, 16, 16)):
+    lib = qmoe.load()
+    arr = (qmoe.qmoe_expert * experts_n)()
+    for i in range(experts_n):
+        arr[i] = qmoe.qmoe_expert(fmt, *ptrs)
+    h = ctypes.c_void_p(12345)
+    st = lib.qmoe_create(ctypes.byref(cfg) if cfg is not None else None, router_w, arr, arr, ctypes.byref(h))
+    return st, h.value
+
+
+@pytest.mark.parametrize("cfg_kw,why", [
+    (dict(d=100, E=8, k=2, I=512, n_shared=0, max_tokens=64), "d"),
+    (dict(d=256, E=8, k=2, I=500, n_shared=0, max_tokens=64), "I"),
+    (dict(d=256, E=0, k=1, I=512, n_shared=0, max_tokens=64), "E"),
+    (dict(d=256, E=300, k=2, I=512, n_shared=0, max_tokens=64), "E"),
+    (dict(d=256, E=8, k=9, I=512, n_shared=0, max_tokens=64), "k"),
+    (dict(d=256, E=32, k=17, I=512, n_shared=0, max_tokens=64), "k"),
+    (dict(d=256, E=8, k=2, I=512, n_shared=9, max_tokens=64), "n_shared"),
+    (dict(d=256, E=8, k=2, I=512, n_shared=0, max_tokens=0), "max_tokens"),
+])
+def test_create_rejects_bad_shapes(cfg_kw, why):
+    cfg = qmoe.qmoe_config(**cfg_kw)
+    st, h = _create_raw(cfg, experts_n=max(1, cfg_kw["E"] + cfg_kw["n_shared"]))
+    assert st == qmoe.QMOE_ERR_INVALID
+    assert h is None
+    assert why in qmoe.qmoe_last_error()
+
+
+def test_create_rejects_null_and_unknown_format():
+    st, _ = _create_raw(None)
+    assert st == qmoe.QMOE_ERR_INVALID
+    cfg = qmoe.qmoe_config(256, 2, 1, 256, 0, 4)
+    st, _ = _create_raw(cfg, experts_n=2, fmt=7)
+    assert st == qmoe.QMOE_ERR_INVALID and "format" in qmoe.qmoe_last_error()
+    st, _ = _create_raw(cfg, experts_n=2, ptrs=(16, None, 16, 16))
+    assert st == qmoe.QMOE_ERR_INVALID and "NULL" in qmoe.qmoe_last_error()
+
+
+def test_calls_reject_null_handle():
+    with pytest.raises(qmoe.QmoeError) as ei:
+        qmoe.qmoe_forward(None, 16, 4, 16)
+    assert ei.value.status == qmoe.QMOE_ERR_INVALID
+    with pytest.raises(qmoe.QmoeError):
+        qmoe.qmoe_route(None, 16, None, 4, 16, 16, 16, 16, 16, 16)
+    with pytest.raises(qmoe.QmoeError):
+        qmoe.qmoe_check_error(None)
