@@ -1,0 +1,442 @@
+"""Throughput of the quantised top-k MoE FFN layer forward on B200.
+
+One step = one qmoe_forward (router, schedule, gate/up GEMM, down GEMM,
+combine) over one batch of seeded synthetic tokens already resident in HBM.
+Default workload: the decode-shaped layer (d=2048, E=128, top-8, I=768, INT4
+group-128 weights) at T=256 tokens, the largest of its token sweep; the
+other sweep points are reported under "sweep".  L2 (126 MB) is flushed by
+writing a 256 MB buffer between timed steps, outside each step's events.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--T T]
+  python bench.py --impl reference ...   # the fp64 CPU oracle on the same workload
+
+Multi-GPU (torchrun, one rank per GPU): the layer does not shard; every rank
+runs an independent replica on its own batch (weak scaling, no collective on
+the data path).  Timing is the max over ranks; value counts all ranks' tokens.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s on 1xB200; % of HBM / tensor-core roofline"
+UNIT = "tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas only)
+# ---------------------------------------------------------------------------
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(backend: str):
+    import torch.distributed as dist
+    world, rank, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank float across the job (identity on one process)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# workload bookkeeping
+# ---------------------------------------------------------------------------
+def workload_desc(L) -> str:
+    from quantized_top_routed_b200 import synth
+    fmts = sorted({synth.FMT_NAMES[ex.fmt] for ex in L.experts})
+    return (f"{L.name} T={L.T} d={L.d} E={L.E} k={L.k} I={L.I} shared={L.S} "
+            f"weights={'+'.join(fmts)}" + (" zipf-bias" if L.router_b is not None else ""))
+
+
+def gate_up_bytes(L, touched) -> int:
+    """Algorithmic HBM bytes of one gate/up GEMM launch: the codes and scales of
+    every touched expert's W13 (and always-on shared experts), the token rows
+    read once and the H rows written once."""
+    wb = sum(L.experts[e].w13.nbytes + L.experts[e].s13.nbytes for e in touched)
+    wb += sum(L.experts[L.E + s].w13.nbytes + L.experts[L.E + s].s13.nbytes for s in range(L.S))
+    return int(wb + L.T * L.d * 2 + L.T * (L.k + L.S) * L.I * 2)
+
+
+def layer_bytes(L, touched) -> int:
+    """Algorithmic HBM bytes of one forward: touched experts' weights and scales,
+    router weights, x read once and out written once."""
+    wb = sum(L.experts[e].w13.nbytes + L.experts[e].s13.nbytes + L.experts[e].w2.nbytes + L.experts[e].s2.nbytes
+             for e in list(touched) + list(range(L.E, L.E + L.S)))
+    return int(wb + L.router_w.nbytes + 4 * L.T * L.d)
+
+
+def gate_up_flops(L) -> float:
+    return 4.0 * L.T * (L.k + L.S) * L.d * L.I
+
+
+def layer_flops(L) -> float:
+    return 2.0 * L.T * L.d * L.E + 6.0 * L.T * (L.k + L.S) * L.d * L.I
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region (NVML, read-only)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def time_steps(fn, steps, warmup, flush, stream):
+    """Per-step CUDA-event times (ms) on `stream`, L2 flushed between steps."""
+    import torch
+    for _ in range(warmup):
+        flush.zero_()
+        fn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in evs:
+        flush.zero_()
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def run_ours(args):
+    import torch
+    import oracle.qmoe_oracle as O  # cpu_baseline leg only
+    from quantized_top_routed_b200 import qmoe, synth
+
+    world, rank = init_dist("nccl")
+    _, _, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks = measured_peaks()
+
+    L = synth.make_layer(args.config, T=args.T, seed=args.seed + rank)
+    dl = qmoe.DeviceLayer(L, max_tokens=L.T, device=str(dev))
+    T = L.T
+    stream = torch.cuda.current_stream()
+    out = torch.empty((T, L.d), dtype=torch.int16, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    # routing of this batch: which experts are touched (bytes never count untouched ones)
+    counts = torch.empty(L.E, dtype=torch.int32, device=dev)
+    scratch = [torch.empty((T, L.k), dtype=torch.int32, device=dev),
+               torch.empty((T, L.k), dtype=torch.float32, device=dev), counts,
+               torch.empty(L.E + 1, dtype=torch.int32, device=dev),
+               torch.empty(T * L.k, dtype=torch.int32, device=dev),
+               torch.empty((T, L.k), dtype=torch.int32, device=dev)]
+    qmoe.qmoe_route(dl.handle, dl.x, None, T, *scratch, stream)
+    torch.cuda.synchronize()
+    cnt = counts.cpu().numpy()
+    touched = [int(e) for e in np.nonzero(cnt)[0]]
+
+    def step():
+        qmoe.qmoe_forward(dl.handle, dl.x, T, out, stream)
+
+    # ---- timed region ------------------------------------------------------
+    barrier(dev)
+    torch.cuda.synchronize()
+    qmoe.qmoe_profile(dl.handle, True)
+    with ClockSampler(local) as clk:
+        times = time_steps(step, args.steps, args.warmup, flush, stream)
+    torch.cuda.synchronize()
+    barrier(dev)
+    stage_ms, calls = qmoe.qmoe_profile_read(dl.handle)
+    qmoe.qmoe_profile(dl.handle, False)
+    qmoe.qmoe_check_error(dl.handle, stream)
+    # warm-up steps were profiled as well; per-launch averages use all calls
+    local_ms = sum(times) / len(times)
+    ms = max_over_ranks(local_ms, dev)
+    value = world * T / (ms / 1e3)
+
+    # ---- end to end through the host-buffer entry point ----------------------
+    x_host = torch.from_numpy(L.x.view(np.int16).copy()).pin_memory()
+    out_host = torch.empty((T, L.d), dtype=torch.int16).pin_memory()
+
+    def e2e_step():
+        qmoe.qmoe_forward_host(dl.handle, x_host, T, out_host, stream)
+
+    barrier(dev)
+    e2e_times = time_steps(e2e_step, args.steps, args.warmup, flush, stream)
+    barrier(dev)
+    e2e_ms = max_over_ranks(sum(e2e_times) / len(e2e_times), dev)
+
+    # ---- roofline of the dominant kernel -----------------------------------
+    gu_ms = stage_ms["gate_up"] / max(calls, 1)
+    hbm_bound = L.name in ("decode", "tiny")
+    if hbm_bound:
+        algo = gate_up_bytes(L, touched)
+        achieved = algo / (gu_ms / 1e3) / 1e9
+        roof = {"kernel": "grouped_gemm gate/up (SwiGLU)", "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": traffic_from_profiles(L, "gate_up"), "peak_source": peaks["source"],
+                "algorithmic_bytes": algo, "avg_launch_ms": round(gu_ms, 5)}
+    else:
+        fl = gate_up_flops(L)
+        achieved = fl / (gu_ms / 1e3) / 1e12
+        peak = peaks["bf16_tflops"]
+        roof = {"kernel": "grouped_gemm gate/up (SwiGLU)", "bound": "tensor", "achieved": round(achieved, 1),
+                "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "traffic": traffic_from_profiles(L, "gate_up"), "peak_source": peaks["source"],
+                "algorithmic_flops": fl, "avg_launch_ms": round(gu_ms, 5)}
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, shapes of the workload)",
+        "config": {"workload": workload_desc(L), "T": T, "global_batch": world * T, "parallelism": f"replicas x{world}",
+                   "l2": "flushed between timed steps (256 MB write)", "touched_experts": len(touched)},
+        "layer": {"bytes": layer_bytes(L, touched), "flops": layer_flops(L),
+                  "hbm_frac": round(layer_bytes(L, touched) / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+                  "tensor_frac": round(layer_flops(L) / (ms / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
+                  "stage_ms": {k_: round(v / max(calls, 1), 5) for k_, v in stage_ms.items()}},
+        "roofline": roof,
+        "e2e": {"value": round(world * T / (e2e_ms / 1e3), 1), "unit": UNIT,
+                "h2d_bytes_per_step": int(T * L.d * 2), "d2h_bytes_per_step": int(T * L.d * 2)},
+        "gpu_launches": qmoe.qmoe_launches_per_forward(dl.handle, T) * args.steps,
+        "clocks": clk.summary(),
+    }
+    if args.sweep and L.name == "decode" and rank == 0:
+        result["sweep"] = sweep_decode(L, dl, flush, stream, peaks)
+    if rank == 0 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(L, O, args)
+    dl.close()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+
+
+def sweep_decode(L, dl, flush, stream, peaks):
+    import dataclasses
+    import torch
+    from quantized_top_routed_b200 import qmoe
+    rows = []
+    for T in (1, 8, 32, 128, 256):
+        if T > L.T:
+            continue
+        sub = dataclasses.replace(L, T=T, x=L.x[:T])
+        out = torch.empty((T, L.d), dtype=torch.int16, device=dl.x.device)
+        xs = dl.x[:T]
+        counts = torch.empty(L.E, dtype=torch.int32, device=dl.x.device)
+        scratch = [torch.empty((T, L.k), dtype=torch.int32, device=dl.x.device),
+                   torch.empty((T, L.k), dtype=torch.float32, device=dl.x.device), counts,
+                   torch.empty(L.E + 1, dtype=torch.int32, device=dl.x.device),
+                   torch.empty(T * L.k, dtype=torch.int32, device=dl.x.device),
+                   torch.empty((T, L.k), dtype=torch.int32, device=dl.x.device)]
+        qmoe.qmoe_route(dl.handle, xs, None, T, *scratch, stream)
+        torch.cuda.synchronize()
+        touched = [int(e) for e in np.nonzero(counts.cpu().numpy())[0]]
+        qmoe.qmoe_profile(dl.handle, True)
+        times = time_steps(lambda: qmoe.qmoe_forward(dl.handle, xs, T, out, stream), 200, 5, flush, stream)
+        stage_ms, calls = qmoe.qmoe_profile_read(dl.handle)
+        qmoe.qmoe_profile(dl.handle, False)
+        ms = sum(times) / len(times)
+        lb = layer_bytes(sub, touched)
+        gu = stage_ms["gate_up"] / max(calls, 1)
+        rows.append({"T": T, "tokens_per_s": round(T / (ms / 1e3), 1), "ms": round(ms, 5),
+                     "touched_experts": len(touched), "layer_hbm_frac": round(lb / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+                     "gate_up_hbm_frac": round(gate_up_bytes(sub, touched) / (gu / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+                     "stage_ms": {k_: round(v / max(calls, 1), 5) for k_, v in stage_ms.items()}})
+    return rows
+
+
+def traffic_from_profiles(L, kernel):
+    """DRAM bytes per launch from a committed ncu summary, if one matches this
+    workload and kernel (profiles/traffic.json), else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    key = f"{L.name}:T={L.T}:{kernel}"
+    v = d.get(key)
+    return None if v is None else v.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# the fp64 oracle, timed on the host cores
+# ---------------------------------------------------------------------------
+def oracle_sample_tokens(L, n, step):
+    return np.array([(step * n + i) % L.T for i in range(n)])
+
+
+def cpu_baseline(L, O, args):
+    from threadpoolctl import threadpool_limits
+    n = args.cpu_tokens
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        O.forward(L, tokens=oracle_sample_tokens(L, n, 0))
+        dt = time.perf_counter() - t0
+    return {"value": round(n / dt, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{n} tokens of the same batch (routing, dequantisation of the touched experts "
+                      f"and the expert FFNs in float64, single thread), {dt:.1f} s"}
+
+
+def oracle_task(O, L, step):
+    """One sampled task of the workload through the oracle: route token t and run
+    the FFN of its slot j (expert-centric task list order), weighted by its gate."""
+    t = step % L.T
+    j = (step // L.T) % L.k
+    r = O.route(L, tokens=[t])
+    e = int(r["idx"][0, j])
+    w13, w2 = O.dequantize_expert(L.experts[e], L.d, L.I)
+    y = O.expert_ffn(O.bf16_to_f64(L.x[t:t + 1]), w13, w2, L.I)
+    return r["gates"][0, j] * y
+
+
+def run_reference(args):
+    """--impl reference: the fp64 CPU oracle, as it stands, on the same workload.
+
+    Each step is one sampled task (a token's routing plus one of its k expert
+    FFNs), so K steps stay within minutes; throughput is scaled to tokens
+    (one task = 1/k token)."""
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle.qmoe_oracle as O
+    from threadpoolctl import threadpool_limits
+    from quantized_top_routed_b200 import synth
+    L = synth.make_layer(args.config, T=args.T, seed=args.seed)
+    with threadpool_limits(limits=1):
+        for w in range(args.warmup):
+            oracle_task(O, L, w)
+        times = []
+        for s in range(args.steps):
+            t0 = time.perf_counter()
+            oracle_task(O, L, args.warmup + s)
+            times.append(time.perf_counter() - t0)
+    ms = 1e3 * sum(times) / len(times)
+    value = (1.0 / L.k) / (ms / 1e3)
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, shapes of the workload)",
+        "config": {"workload": workload_desc(L), "T": L.T, "sample": "one routed task (1/k token) per step"},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": "per step one token's routing and one of its k expert FFNs in float64, "
+                                   "single thread; tokens/s = (1/k) / step time"},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--config", default="decode", choices=("tiny", "decode", "prefill", "fine", "mixed"))
+    ap.add_argument("--T", type=int, default=None, help="tokens per step (default: the workload's)")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-sweep", dest="sweep", action="store_false")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-tokens", type=int, default=16, help="tokens in the timed oracle sample")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -10,6 +10,7 @@ from __future__ import annotations
 
 import argparse
 import concurrent.futures
+import hashlib
 import os
 import shutil
 import subprocess
@@ -41,11 +42,26 @@ def _inputs():
     return deps
 
 
+HASH = LIB + ".srchash"
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    for p in _inputs():
+        with open(p, "rb") as f:
+            h.update(os.path.basename(p).encode())
+            h.update(f.read())
+    h.update(" ".join(ARCH + FLAGS).encode())
+    return h.hexdigest()
+
+
 def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+    """The library exists and was built from exactly the current sources
+    (content hash, so copies of the tree with fresh timestamps still match)."""
+    if not (os.path.exists(LIB) and os.path.exists(HASH)):
         return False
-    t = os.path.getmtime(LIB)
-    return all(os.path.getmtime(p) <= t for p in _inputs())
+    with open(HASH) as f:
+        return f.read().strip() == source_hash()
 
 
 def _compile(src: str, verbose: bool) -> str:
@@ -73,6 +89,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
     os.replace(tmp, LIB)
+    with open(HASH, "w") as f:
+        f.write(source_hash())
     return LIB
 
 

@@ -3,6 +3,7 @@
 //   router logits -> router top-k -> schedule -> gate/up GEMM -> down GEMM -> combine
 // on the caller's stream.  No call synchronises the stream on the hot path;
 // the counts never travel to the host (the GEMMs read the device tile tables).
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -40,6 +41,38 @@ struct Event {
   int stage = 0;
 };
 
+// cuTensorMapEncodeTiled, fetched from the driver through the runtime so the
+// library does not link libcuda directly.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// Row-major bf16 matrix [rows][cols] read in 4-row x 64-column gathers into
+// 128-byte-swizzled shared memory.
+bool encode_rows_map(CUtensorMap* m, const void* base, int rows, int cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {64, 1};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 struct qmoe_handle {
@@ -52,8 +85,11 @@ struct qmoe_handle {
   ExpertDev* d_experts = nullptr;
   // workspace
   int32_t *idx = nullptr, *inv_pos = nullptr, *counts = nullptr, *offsets = nullptr, *sorted_token = nullptr;
-  int32_t *seg_off = nullptr, *seg_cnt = nullptr, *tile3 = nullptr, *tile4 = nullptr, *sched_scratch = nullptr;
+  int32_t *seg_off = nullptr, *seg_cnt = nullptr, *tiles = nullptr, *seg_fmt = nullptr, *sched_scratch = nullptr;
+  bool fmt_present[4] = {false, false, false, false};
+  CUtensorMap h_map;                     // H rows for the down GEMM's gathers
   float *gates = nullptr, *zpart = nullptr;
+  int* tickets = nullptr;
   uint16_t *H = nullptr, *Y = nullptr, *x_stage = nullptr, *out_stage = nullptr;
   int* err = nullptr;
   int zpart_split_max = 1;
@@ -146,22 +182,21 @@ qmoe_status route_impl(qmoe_handle* h, const uint16_t* x, const float* logits, i
   const qmoe_config& c = h->cfg;
   {
     StageTimer tm(h, s, QMOE_STAGE_ROUTER);
-    const float* zp = logits;
-    int split = 1;
     if (x) {
-      split = router_split(T, c.d, c.E, h->num_sms);
+      int split = router_split(T, c.d, c.E, h->num_sms);
       if (split > h->zpart_split_max) split = h->zpart_split_max;
-      QMOE_CUDA(launch_router_logits(x, h->router_w, T, c.d, c.E, split, h->zpart, s), "router logits launch");
-      zp = h->zpart;
+      QMOE_CUDA(launch_router(x, h->router_w, h->router_b, T, c.d, c.E, c.k, split, h->zpart, h->tickets, idx,
+                              gates, s),
+                "router launch");
+    } else {
+      QMOE_CUDA(launch_router_topk(logits, T, c.E, c.k, idx, gates, s), "router top-k launch");
     }
-    QMOE_CUDA(launch_router_topk(zp, split, x ? h->router_b : nullptr, T, c.E, c.k, idx, gates, s),
-              "router top-k launch");
   }
   {
     StageTimer tm(h, s, QMOE_STAGE_SCHEDULE);
-    QMOE_CUDA(launch_schedule(idx, T, c.k, c.E, tables ? c.n_shared : 0, bn, 2 * c.I / kTileM, bn, c.d / kTileM,
-                              counts, offsets, sorted_token, inv_pos, tables ? h->seg_off : nullptr,
-                              tables ? h->seg_cnt : nullptr, h->tile3, h->tile4, h->sched_scratch, s),
+    QMOE_CUDA(launch_schedule(idx, T, c.k, c.E, tables ? c.n_shared : 0, bn, 2 * c.I / kTileM, c.d / kTileM,
+                              h->seg_fmt, counts, offsets, sorted_token, inv_pos, tables ? h->seg_off : nullptr,
+                              tables ? h->seg_cnt : nullptr, h->tiles, h->sched_scratch, s),
               "schedule launch");
   }
   return QMOE_OK;
@@ -271,18 +306,33 @@ qmoe_status qmoe_create(const qmoe_config* cfg, const float* router_w, const flo
   if ((st = h->alloc(&h->sorted_token, P, "sorted_token")) != QMOE_OK) return bail(st);
   if ((st = h->alloc(&h->seg_off, (size_t)n_seg, "seg_off")) != QMOE_OK) return bail(st);
   if ((st = h->alloc(&h->seg_cnt, (size_t)n_seg, "seg_cnt")) != QMOE_OK) return bail(st);
-  if ((st = h->alloc(&h->tile3, (size_t)n_seg + 1, "tile3")) != QMOE_OK) return bail(st);
-  if ((st = h->alloc(&h->tile4, (size_t)n_seg + 1, "tile4")) != QMOE_OK) return bail(st);
+  if ((st = h->alloc(&h->tiles, (size_t)6 * (n_seg + 1), "tile tables")) != QMOE_OK) return bail(st);
+  {
+    std::vector<int32_t> fm(n_seg);
+    for (int e = 0; e < n_seg; ++e) {
+      fm[e] = experts[e].fmt;
+      h->fmt_present[experts[e].fmt] = true;
+    }
+    if ((st = h->alloc(&h->seg_fmt, (size_t)n_seg, "segment formats")) != QMOE_OK) return bail(st);
+    if (cudaMemcpy(h->seg_fmt, fm.data(), sizeof(int32_t) * n_seg, cudaMemcpyHostToDevice) != cudaSuccess)
+      return bail(cuda_fail(cudaGetLastError(), "copy segment formats"));
+  }
   if ((st = h->alloc(&h->sched_scratch, schedule_scratch_ints(c.max_tokens, c.E), "schedule scratch")) != QMOE_OK)
     return bail(st);
   if ((st = h->alloc(&h->zpart, (size_t)h->zpart_split_max * Tm * c.E, "router partials")) != QMOE_OK)
     return bail(st);
   if ((st = h->alloc(&h->H, P * c.I, "H")) != QMOE_OK) return bail(st);
+  if (!encode_rows_map(&h->h_map, h->H, (int)P, c.I))
+    return bail(fail(QMOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the H buffer"));
   if ((st = h->alloc(&h->Y, P * c.d, "Y")) != QMOE_OK) return bail(st);
   if ((st = h->alloc(&h->x_stage, Tm * c.d, "x staging")) != QMOE_OK) return bail(st);
   if ((st = h->alloc(&h->out_stage, Tm * c.d, "out staging")) != QMOE_OK) return bail(st);
   if ((st = h->alloc(&h->err, 1, "error word")) != QMOE_OK) return bail(st);
   if (cudaMemset(h->err, 0, sizeof(int)) != cudaSuccess) return bail(cuda_fail(cudaGetLastError(), "memset"));
+  const int ntick = router_tickets(c.max_tokens);
+  if ((st = h->alloc(&h->tickets, (size_t)ntick, "router tickets")) != QMOE_OK) return bail(st);
+  if (cudaMemset(h->tickets, 0, sizeof(int) * ntick) != cudaSuccess)
+    return bail(cuda_fail(cudaGetLastError(), "memset"));
   cudaError_t se = cudaDeviceSynchronize();
   if (se != cudaSuccess) return bail(cuda_fail(se, "qmoe_create"));
   *out = h;
@@ -315,37 +365,30 @@ qmoe_status qmoe_forward(qmoe_handle* h, const uint16_t* x, int32_t T, uint16_t*
   st = route_impl(h, x, nullptr, T, h->idx, h->gates, h->counts, h->offsets, h->sorted_token, h->inv_pos, true, bn, s);
   if (st != QMOE_OK) return st;
 
+  CUtensorMap x_map;
+  if (!encode_rows_map(&x_map, x, T, c.d)) return fail(QMOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for x");
   GemmArgs g{};
   g.experts = h->d_experts;
   g.seg_off = h->seg_off;
   g.seg_cnt = h->seg_cnt;
   g.n_seg = c.E + c.n_shared;
   g.err = h->err;
-  {
-    StageTimer tm(h, s, QMOE_STAGE_GATE_UP);
-    g.mat = 0;
-    g.act = x;
-    g.act_ld = c.d;
-    g.gather = h->sorted_token;
-    g.tile_off = h->tile3;
-    g.K = c.d;
-    g.MB = 2 * c.I / kTileM;
-    g.out = h->H;
-    g.out_ld = c.I;
-    QMOE_CUDA(launch_grouped_gemm(g, bn, h->num_sms, s), "gate/up GEMM launch");
-  }
-  {
-    StageTimer tm(h, s, QMOE_STAGE_DOWN);
-    g.mat = 1;
-    g.act = h->H;
-    g.act_ld = c.I;
-    g.gather = nullptr;
-    g.tile_off = h->tile4;
-    g.K = c.I;
-    g.MB = c.d / kTileM;
-    g.out = h->Y;
-    g.out_ld = c.d;
-    QMOE_CUDA(launch_grouped_gemm(g, bn, h->num_sms, s), "down GEMM launch");
+  for (int mat = 0; mat < 2; ++mat) {
+    StageTimer tm(h, s, mat == 0 ? QMOE_STAGE_GATE_UP : QMOE_STAGE_DOWN);
+    g.mat = mat;
+    g.act = mat == 0 ? x : h->H;
+    g.act_ld = mat == 0 ? c.d : c.I;
+    g.gather = mat == 0 ? h->sorted_token : nullptr;
+    g.K = mat == 0 ? c.d : c.I;
+    g.MB = mat == 0 ? 2 * c.I / kTileM : c.d / kTileM;
+    g.out = mat == 0 ? h->H : h->Y;
+    g.out_ld = mat == 0 ? c.I : c.d;
+    for (int fmt = 1; fmt <= 3; ++fmt) {   // one launch per weight format present
+      if (!h->fmt_present[fmt]) continue;
+      g.tile_off = h->tiles + tile_table_offset(mat, fmt, g.n_seg);
+      QMOE_CUDA(launch_grouped_gemm(g, mat == 0 ? x_map : h->h_map, fmt, bn, h->num_sms, s),
+                mat == 0 ? "gate/up GEMM launch" : "down GEMM launch");
+    }
   }
   {
     StageTimer tm(h, s, QMOE_STAGE_COMBINE);
@@ -405,9 +448,11 @@ qmoe_status qmoe_profile_read(qmoe_handle* h, float* ms, int32_t n, int32_t* cal
 }
 
 int32_t qmoe_launches_per_forward(const qmoe_handle* h, int32_t T) {
-  (void)h;
   (void)T;
-  return 6;  // router logits, router top-k, schedule, gate/up GEMM, down GEMM, combine
+  if (!h) return 0;
+  int fmts = 0;
+  for (int f = 1; f <= 3; ++f) fmts += h->fmt_present[f] ? 1 : 0;
+  return 3 + 2 * fmts;  // router (logits + top-k), schedule, gate/up and down GEMM per format, combine
 }
 
 qmoe_status qmoe_destroy(qmoe_handle* h) {

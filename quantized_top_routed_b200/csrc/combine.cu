@@ -6,8 +6,8 @@
 // active for every input; "FineRMoE", Sparse Sum Layer: outputs weighted by
 // the router's probabilities.)
 //
-// One CTA per token; each thread moves 16-byte vectors (8 bf16), so every Y
-// row and the output row are read/written with coalesced 16-byte accesses.
+// Each thread moves one 16-byte vector (8 bf16) of one token, so every Y row
+// and the output row are read and written with coalesced 16-byte accesses.
 #include "qmoe_internal.cuh"
 
 namespace qmoe {
@@ -27,42 +27,49 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&p);
 }
 
-__global__ void __launch_bounds__(128) combine_kernel(const uint16_t* __restrict__ Y, const float* __restrict__ gate,
+// One thread per 16-byte output vector: all k + S row loads are issued
+// before any accumulation, so a token costs one memory round trip.
+__global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ Y, const float* __restrict__ gate,
                                                       const int32_t* __restrict__ inv_pos, int T, int k, int S,
                                                       int d, uint16_t* __restrict__ out) {
-  __shared__ float g[kMaxK];
-  __shared__ int32_t pos[kMaxK];
-  const int t = blockIdx.x;
-  if (threadIdx.x < k) {
-    g[threadIdx.x] = gate[(size_t)t * k + threadIdx.x];
-    pos[threadIdx.x] = inv_pos[(size_t)t * k + threadIdx.x];
-  }
-  __syncthreads();
   const int nvec = d >> 3;
-  for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
-    float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j < k; ++j) {
-      const uint4 y = __ldg(reinterpret_cast<const uint4*>(Y + (size_t)pos[j] * d) + v);
-      acc8(a, y, g[j]);
+  const long long gv = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gv >= (long long)T * nvec) return;
+  const int t = (int)(gv / nvec), v = (int)(gv - (long long)t * nvec);
+  uint4 y[kMaxK + kMaxShared];
+  float g[kMaxK];
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) {
+    if (j < k) {
+      const int pos = __ldg(inv_pos + (size_t)t * k + j);
+      g[j] = __ldg(gate + (size_t)t * k + j);
+      y[j] = __ldg(reinterpret_cast<const uint4*>(Y + (size_t)pos * d) + v);
     }
-    for (int s = 0; s < S; ++s) {
-      const uint4 y = __ldg(reinterpret_cast<const uint4*>(Y + ((size_t)T * k + (size_t)s * T + t) * d) + v);
-      acc8(a, y, 1.0f);
-    }
-    uint4 o;
-    o.x = pack_bf16x2(a[0], a[1]);
-    o.y = pack_bf16x2(a[2], a[3]);
-    o.z = pack_bf16x2(a[4], a[5]);
-    o.w = pack_bf16x2(a[6], a[7]);
-    reinterpret_cast<uint4*>(out + (size_t)t * d)[v] = o;
   }
+#pragma unroll
+  for (int s = 0; s < kMaxShared; ++s)
+    if (s < S) y[kMaxK + s] = __ldg(reinterpret_cast<const uint4*>(Y + ((size_t)T * k + (size_t)s * T + t) * d) + v);
+  float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j)
+    if (j < k) acc8(a, y[j], g[j]);
+#pragma unroll
+  for (int s = 0; s < kMaxShared; ++s)
+    if (s < S) acc8(a, y[kMaxK + s], 1.0f);
+  uint4 o;
+  o.x = pack_bf16x2(a[0], a[1]);
+  o.y = pack_bf16x2(a[2], a[3]);
+  o.z = pack_bf16x2(a[4], a[5]);
+  o.w = pack_bf16x2(a[6], a[7]);
+  reinterpret_cast<uint4*>(out + (size_t)t * d)[v] = o;
 }
 
 }  // namespace
 
 cudaError_t launch_combine(const uint16_t* Y, const float* gate, const int32_t* inv_pos, int T, int k, int S, int d,
                            uint16_t* out, cudaStream_t s) {
-  combine_kernel<<<T, 128, 0, s>>>(Y, gate, inv_pos, T, k, S, d, out);
+  const long long n = (long long)T * (d >> 3);
+  combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(Y, gate, inv_pos, T, k, S, d, out);
   return cudaGetLastError();
 }
 

@@ -13,52 +13,78 @@
 //   A (M x K) = 128 weight rows, dequantised to bf16 by CUDA cores and
 //               written straight into tensor memory (tcgen05.st);
 //   B (N x K) = up to BN rows of the expert's segment (tokens), gathered
-//               from x / H into 128-byte-swizzled shared memory (cp.async);
+//               from x / H by TMA (tile::gather4) into 128-byte-swizzled
+//               shared memory;
 //   D (M x N) = fp32 accumulators in tensor memory, double buffered.
-// Weights are the M side because an expert usually has few tokens; the
-// weight stream is what the kernel moves.  INT4 group scales are applied
+// Weights are the M side because an expert usually has few tokens: the
+// weight stream is what the kernel moves.  Raw code tiles arrive by TMA bulk
+// copy into a ring sized per weight format (no instruction cost per byte);
+// the dequantisation warps read them with conflict-free 16-byte shared
+// loads.  Every role signals once per warp per stage, so the SM's issue
+// slots go to the dequantisation arithmetic.  INT4 group scales are applied
 // during dequantisation (bf16(q*s), one rounding); INT8 and FP8 per-channel
 // scales are applied to the fp32 accumulator in the epilogue (exact
 // factoring).
 //
 // Persistent CTAs (one per SM) walk the tile list (segment, 128-row weight
-// block, BN-row token block) built on the device by the schedule kernel.
-// Warp roles, all synchronised through mbarriers:
-//   warp 0      : TMEM allocation; lane 0 streams raw weight tiles (bulk copy)
-//   warp 1      : lane 0 issues the MMAs and the commits
-//   warps 2..5  : gather the B rows (cp.async) and dequantise A into TMEM
-//   warps 6..9  : epilogue (TMEM -> registers -> scales / SwiGLU -> bf16)
+// block, BN-row token block) built on the device by the schedule kernel;
+// one launch handles the experts of one weight format.  Warp roles, all
+// synchronised through mbarriers:
+//   warp 0       : TMEM allocation; lane 0 streams raw weight tiles (bulk copy)
+//   warp 1       : lanes issue the B gathers (TMA tile::gather4)
+//   warp 2       : lane 0 issues the MMAs and the commits
+//   warps 3..10  : dequantise A into TMEM; warp w owns TMEM lane quarter
+//                  w % 4 and one 64-wide half of every 128-wide K stage
+//   warps 11..14 : epilogue (TMEM -> registers -> scales / SwiGLU -> bf16)
 // Every wait is bounded: a role that waits ~1 s raises an abort flag, all
 // roles drain what they issued, TMEM is freed and the error word is set.
+#include <cuda.h>
+
+#include <type_traits>
+
 #include "qmoe_internal.cuh"
 
 namespace qmoe {
 namespace {
 
-constexpr int kThreads = 320;
-constexpr int kRawSlot = 16384;
+constexpr int kNDQ = 8;                        // dequantisation warps
+constexpr int kKW = kBK / (kNDQ / 4);          // K elements one dequant thread converts per stage (64)
+constexpr int kRawWarp = 0, kBWarp = 1, kMmaWarp = 2;
+constexpr int kDQWarp0 = 3;
+constexpr int kEpiWarp0 = kDQWarp0 + kNDQ;
+constexpr int kThreads = 32 * (kEpiWarp0 + 4);
 constexpr int kTabMax = kMaxE + kMaxShared + 1;
 constexpr uint32_t kTmemCols = 512;
 
-template <int BN>
+template <int FMT>
+struct FmtCfg {
+  static constexpr int SB = FMT == QMOE_W_INT4_G128 ? 128 * 64 + 256 : 128 * 128;  // bytes of a raw tile
+  static constexpr int NC = FMT == QMOE_W_INT4_G128 ? kKW / 32 : kKW / 16;          // 16-byte chunks per thread
+};
+
+template <int BN, int FMT>
 struct Cfg {
   static constexpr int SA = BN >= 128 ? 4 : (BN >= 64 ? 6 : 7);   // A/B stages (TMEM + smem)
-  static constexpr int R = BN >= 128 ? 3 : (BN >= 64 ? 6 : 8);    // raw weight ring
   static constexpr int B_STAGE = BN * 256;                        // BN rows x 128 K bf16
   static constexpr int STAGING = BN * 256;                        // epilogue staging
   static constexpr int A_COL0 = 2 * BN;                           // TMEM: acc0, acc1, then A stages
+  static constexpr int SLOT = (FmtCfg<FMT>::SB + 127) & ~127;     // raw ring slot
+  static constexpr int FIXED = SA * B_STAGE + STAGING + 6 * 1024;
+  static constexpr int R0 = (224 * 1024 - FIXED) / SLOT;
+  static constexpr int R = R0 > 16 ? 16 : R0;                     // raw ring depth
   static constexpr int OFF_B = 0;
   static constexpr int OFF_RAW = OFF_B + SA * B_STAGE;
-  static constexpr int OFF_STG = OFF_RAW + R * kRawSlot;
+  static constexpr int OFF_STG = OFF_RAW + R * SLOT;
   static constexpr int OFF_TAB = OFF_STG + STAGING;
-  static constexpr int OFF_BAR = (OFF_TAB + 3 * kTabMax * 4 + 127) & ~127;  // mbarriers: 8-byte aligned
+  static constexpr int OFF_BAR = (OFF_TAB + 3 * kTabMax * 4 + 127) & ~127;
   static constexpr int NUM_BARS = 2 * SA + 2 * R + 4 + 1;
   static constexpr int OFF_MISC = (OFF_BAR + NUM_BARS * 8 + 15) & ~15;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;               // + alignment slack
-  static_assert(OFF_BAR % 8 == 0 && OFF_MISC % 16 == 0, "barrier alignment");
-  static_assert(OFF_RAW % 1024 == 0 && OFF_STG % 16 == 0 && B_STAGE % 1024 == 0, "buffer alignment");
+  static_assert(R >= 3, "raw ring too shallow");
   static_assert(A_COL0 + SA * 64 <= (int)kTmemCols, "TMEM budget");
   static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(B_STAGE % 1024 == 0 && OFF_RAW % 1024 == 0 && OFF_BAR % 8 == 0 && OFF_MISC % 16 == 0,
+                "alignment");
 };
 
 struct Tile {
@@ -84,7 +110,7 @@ __device__ __forceinline__ Tile decode_tile(int tile, const int32_t* tab_off, co
   return t;
 }
 
-// ---- dequantisation to bf16 pairs ------------------------------------------
+// ---- dequantisation ----------------------------------------------------------
 __device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t mask, uint32_t orv) {
   return (a & mask) | orv;
 }
@@ -123,6 +149,31 @@ __device__ __forceinline__ void deq_fp8_word(uint32_t w, uint32_t* o) {
   o[1] = bf2_mul(hi, 0x7B807B80u);
 }
 
+// This thread's 16-byte chunks (K order) -> kKW / 2 bf16 pairs.
+template <int FMT>
+__device__ __forceinline__ void dequant_slice(const uint4 (&w)[FmtCfg<FMT>::NC], uint32_t sbits, uint32_t* av) {
+#pragma unroll
+  for (int c = 0; c < FmtCfg<FMT>::NC; ++c) {
+    if constexpr (FMT == QMOE_W_INT4_G128) {
+      const uint32_t s2 = sbits | (sbits << 16);
+      deq_int4_word(w[c].x, s2, &av[16 * c + 0]);
+      deq_int4_word(w[c].y, s2, &av[16 * c + 4]);
+      deq_int4_word(w[c].z, s2, &av[16 * c + 8]);
+      deq_int4_word(w[c].w, s2, &av[16 * c + 12]);
+    } else if constexpr (FMT == QMOE_W_FP8_E4M3_PC) {
+      deq_fp8_word(w[c].x, &av[8 * c + 0]);
+      deq_fp8_word(w[c].y, &av[8 * c + 2]);
+      deq_fp8_word(w[c].z, &av[8 * c + 4]);
+      deq_fp8_word(w[c].w, &av[8 * c + 6]);
+    } else {
+      deq_int8_word(w[c].x, &av[8 * c + 0]);
+      deq_int8_word(w[c].y, &av[8 * c + 2]);
+      deq_int8_word(w[c].z, &av[8 * c + 4]);
+      deq_int8_word(w[c].w, &av[8 * c + 6]);
+    }
+  }
+}
+
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
 
 __device__ __forceinline__ uint16_t f2bf(float f) {
@@ -130,11 +181,29 @@ __device__ __forceinline__ uint16_t f2bf(float f) {
   return *reinterpret_cast<const uint16_t*>(&b);
 }
 
-template <int BN, int MAT>
-__global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArgs a) {
-  using C = Cfg<BN>;
+// TMA: 4 rows (arbitrary row indices) x 64 bf16 columns of a row-major
+// matrix into 512 bytes of 128-byte-swizzled shared memory.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, int col, int r0, int r1, int r2,
+                                            int r3, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Warp-uniform bounded wait: every lane polls, the warp proceeds together.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
+}
+
+template <int BN, int MAT, int FMT>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap act_map) {
+  using C = Cfg<BN, FMT>;
+  using F = FmtCfg<FMT>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sB = smem + C::OFF_B;
   uint8_t* sRaw = smem + C::OFF_RAW;
   uint8_t* sStg = smem + C::OFF_STG;
@@ -142,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
   int32_t* s_seg_off = tab_off + kTabMax;
   int32_t* s_seg_cnt = s_seg_off + kTabMax;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* full = bars;                      // [SA] B gathered + A in TMEM
+  uint64_t* full = bars;                      // [SA] B landed + A in TMEM
   uint64_t* empty = full + C::SA;             // [SA] MMA done with stage
   uint64_t* raw_full = empty + C::SA;         // [R] raw tile landed
   uint64_t* raw_empty = raw_full + C::R;      // [R] raw tile consumed
@@ -165,47 +234,46 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
   }
   if (tid == 0) {
     for (int s = 0; s < C::SA; ++s) {
-      mbar_init(&full[s], 256);
+      mbar_init(&full[s], 1 + kNDQ);   // B producer expect_tx + one arrival per dequant warp
       mbar_init(&empty[s], 1);
     }
     for (int r = 0; r < C::R; ++r) {
       mbar_init(&raw_full[r], 1);
-      mbar_init(&raw_empty[r], 128);
+      mbar_init(&raw_empty[r], kNDQ);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 128);
+      mbar_init(&acc_empty[b], 4);     // one arrival per epilogue warp
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
+  if (warp == kRawWarp) tmem_alloc(tmem_slot, kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total = tab_off[n_seg];
 
-  if (warp == 0) {
-    // ---------------- raw weight producer ----------------
-    uint32_t rc = 0;
+  if (warp == kRawWarp) {
+    // ---------------- raw weight tiles: one bulk copy per K stage ----------------
+    uint32_t rc = 0, r = 0, ph = 0;         // copies issued, ring slot, slot parity
     bool ok = true;
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
       const Tile t = decode_tile(tile, tab_off, s_seg_off, s_seg_cnt, n_seg, BN);
-      const ExpertDev& ex = a.experts[t.seg];
-      const int sb = stage_bytes(ex.fmt);
-      const uint8_t* src = ex.w[MAT] + (size_t)t.mb * KS * sb;
+      const uint8_t* src = a.experts[t.seg].w[MAT] + (size_t)t.mb * KS * F::SB;
       for (int ks = 0; ks < KS; ++ks) {
-        const int slot = rc % C::R;
-        ok = __all_sync(0xffffffffu, mbar_wait(&raw_empty[slot], ((rc / C::R) & 1) ^ 1, abort_flag));
+        ok = warp_wait(&raw_empty[r], ph ^ 1, abort_flag);
         if (!ok) break;
         if (lane == 0) {
-          mbar_arrive_expect_tx(&raw_full[slot], sb);
-          bulk_g2s(sRaw + slot * kRawSlot, src + (size_t)ks * sb, sb, &raw_full[slot]);
+          mbar_arrive_expect_tx(&raw_full[r], F::SB);
+          bulk_g2s(sRaw + r * C::SLOT, src, F::SB, &raw_full[r]);
         }
-        ++rc;
         __syncwarp();
+        src += F::SB;
+        ++rc;
+        if (++r == (uint32_t)C::R) { r = 0; ph ^= 1; }
       }
     }
     // wait for copies that may still be in flight before the CTA can exit
@@ -214,36 +282,72 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
       for (uint32_t i = first; i < rc; ++i) mbar_wait_drain(&raw_full[i % C::R], (i / C::R) & 1);
     }
     __syncwarp();
-  } else if (warp == 1) {
+  } else if (warp == kBWarp) {
+    // ---------------- B rows: TMA gathers of the tile's tokens ----------------
+    uint32_t sc = 0, s = 0, ph = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      const Tile t = decode_tile(tile, tab_off, s_seg_off, s_seg_cnt, n_seg, BN);
+      const int groups = (t.nvalid + 3) >> 2;            // 4-row gathers per K atom
+      int rr[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {                       // lane l gathers rows 4l .. 4l+3
+        const int n = 4 * lane + j;
+        const int p = t.row0 + (n < t.nvalid ? n : 0);
+        rr[j] = (lane < groups) ? (a.gather ? a.gather[p] : p) : 0;
+      }
+      for (int ks = 0; ks < KS; ++ks) {
+        ok = warp_wait(&empty[s], ph ^ 1, abort_flag);
+        if (!ok) break;
+        if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)groups * 4 * 256);
+        __syncwarp();
+        if (lane < groups) {
+          const uint32_t dst = smem_u32(sB + s * C::B_STAGE) + lane * 512;
+          tma_gather4(dst, &act_map, ks * kBK, rr[0], rr[1], rr[2], rr[3], &full[s]);
+          tma_gather4(dst + BN * 128, &act_map, ks * kBK + 64, rr[0], rr[1], rr[2], rr[3], &full[s]);
+        }
+        __syncwarp();
+        ++sc;
+        if (++s == (uint32_t)C::SA) { s = 0; ph ^= 1; }
+      }
+    }
+    if (lane == 0) {
+      const uint32_t first = sc > (uint32_t)C::SA ? sc - C::SA : 0;
+      for (uint32_t i = first; i < sc; ++i) mbar_wait_drain(&full[i % C::SA], (i / C::SA) & 1);
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
-    uint32_t sc = 0, tc = 0;
+    uint32_t s = 0, ph = 0, tc = 0;
+    const uint64_t bdesc0 = smem_desc_sw128(smem_u32(sB));
+    const uint32_t a_tmem0 = tmem_base + C::A_COL0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++tc) {
       const Tile t = decode_tile(tile, tab_off, s_seg_off, s_seg_cnt, n_seg, BN);
       const int b = tc & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(&acc_empty[b], ((tc >> 1) & 1) ^ 1, abort_flag));
+      ok = warp_wait(&acc_empty[b], ((tc >> 1) & 1) ^ 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
       const int n_mma = max(16, (t.nvalid + 15) & ~15);
       const uint32_t idesc = idesc_bf16_m128(n_mma);
       const uint32_t d_tmem = tmem_base + b * BN;
-      for (int ks = 0; ks < KS; ++ks, ++sc) {
-        const int s = sc % C::SA;
-        ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (sc / C::SA) & 1, abort_flag));
+      for (int ks = 0; ks < KS; ++ks) {
+        ok = warp_wait(&full[s], ph, abort_flag);
         if (!ok) break;
         tc_fence_after();
         if (lane == 0) {
-          fence_proxy_async_smem();
-          const uint32_t bbase = smem_u32(sB + s * C::B_STAGE);
+          // Descriptors of this stage: only the start-address field moves
+          // (16-byte units), so each MMA's operands are one add away.
+          const uint64_t bdesc = bdesc0 + (uint64_t)(s * (C::B_STAGE >> 4));
+          const uint32_t a_tmem = a_tmem0 + s * 64;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t a_tmem = tmem_base + C::A_COL0 + s * 64 + kk * 8;
-            const uint64_t bdesc = smem_desc_sw128(bbase + (kk >> 2) * (BN * 128) + (kk & 3) * 32);
-            mma_bf16_ts(d_tmem, a_tmem, bdesc, idesc, (ks | kk) != 0);
-          }
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ts(d_tmem, a_tmem + kk * 8, bdesc + (uint64_t)((kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2),
+                        idesc, (ks | kk) != 0);
           mma_commit(&empty[s]);
         }
         __syncwarp();
+        if (++s == (uint32_t)C::SA) { s = 0; ph ^= 1; }
       }
       if (!ok) break;
       if (lane == 0) mma_commit(&acc_full[b]);
@@ -257,106 +361,54 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
       }
       __syncwarp();
     }
-  } else if (warp < 6) {
-    // ---------------- B gather + A dequantisation ----------------
-    const int dq = tid - 64;                 // 0..127
-    const int q = warp & 3;                  // TMEM lane quarter
-    const int r = 32 * q + lane;             // weight row of the tile
-    const int ch = dq & 15;                  // 16-byte chunk of a 256-byte B row
-    const int katom = ch >> 3, cc = ch & 7;
-    constexpr int RPT = BN / 8;              // B rows per thread
-    uint32_t sc = 0, rc = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-      const Tile t = decode_tile(tile, tab_off, s_seg_off, s_seg_cnt, n_seg, BN);
-      const int fmt = a.experts[t.seg].fmt;
-      const uint16_t* srcp[RPT];
-      uint32_t srcn[RPT];
+  } else if (warp < kEpiWarp0) {
+    // ---------------- A dequantisation into TMEM ----------------
+    const int q = warp & 3;                          // TMEM lane quarter
+    const int h = (warp - kDQWarp0) >> 2;            // which half of the K stage
+    const int row = 32 * q + lane;                   // weight row of the tile
+    const uint32_t coff = (uint32_t)(h * F::NC) * 2048u + (uint32_t)row * 16u;   // chunk-major raw tile
+    const uint32_t soff = 128u * 64u + (uint32_t)row * 2u;                       // INT4 group scale
+    const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + C::A_COL0 + h * (kKW / 2);
+    const uint32_t raw0 = smem_u32(sRaw);
+    uint32_t s = 0, ph = 0, r = 0, rph = 0;
+    int left = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) left += KS;
+    while (left > 0) {
+      if (!warp_wait(&raw_full[r], rph, abort_flag)) break;
+      const uint32_t rp = raw0 + r * C::SLOT;
+      uint4 w[F::NC];
 #pragma unroll
-      for (int i = 0; i < RPT; ++i) {
-        const int n = (dq >> 4) + 8 * i;
-        if (n < t.nvalid) {
-          const int row = a.gather ? a.gather[t.row0 + n] : t.row0 + n;
-          srcp[i] = a.act + (size_t)row * a.act_ld + ch * 8;
-          srcn[i] = 16;
-        } else {
-          srcp[i] = a.act;
-          srcn[i] = 0;
-        }
+      for (int k = 0; k < F::NC; ++k)
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w[k].x), "=r"(w[k].y), "=r"(w[k].z), "=r"(w[k].w)
+                     : "r"(rp + coff + k * 2048));
+      uint32_t sbits = 0;
+      if constexpr (FMT == QMOE_W_INT4_G128) {
+        unsigned short sv;
+        asm volatile("ld.shared.u16 %0, [%1];" : "=h"(sv) : "r"(rp + soff));
+        sbits = sv;
       }
-      for (int ks = 0; ks < KS; ++ks, ++sc, ++rc) {
-        const int s = sc % C::SA;
-        ok = __all_sync(0xffffffffu, mbar_wait(&empty[s], ((sc / C::SA) & 1) ^ 1, abort_flag));
-        if (!ok) break;
-        const uint32_t bst = smem_u32(sB + s * C::B_STAGE) + katom * (BN * 128);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&raw_empty[r]);
+      if (++r == (uint32_t)C::R) { r = 0; rph ^= 1; }
+      uint32_t av[kKW / 2];
+      dequant_slice<FMT>(w, sbits, av);
+      if (!warp_wait(&empty[s], ph ^ 1, abort_flag)) break;
 #pragma unroll
-        for (int i = 0; i < RPT; ++i) {
-          const int n = (dq >> 4) + 8 * i;
-          cp_async16(bst + n * 128 + ((cc ^ (n & 7)) << 4), srcp[i] + (size_t)ks * kBK, srcn[i]);
-        }
-        cp_async_arrive_noinc(&full[s]);
-
-        const int slot = rc % C::R;
-        ok = __all_sync(0xffffffffu, mbar_wait(&raw_full[slot], (rc / C::R) & 1, abort_flag));
-        if (!ok) break;
-        const uint8_t* rawp = sRaw + slot * kRawSlot;
-        uint32_t av[64];
-        if (fmt == QMOE_W_INT4_G128) {
-          uint4 wv[4];
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            wv[c] = *reinterpret_cast<const uint4*>(rawp + r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
-          const uint32_t sbits = reinterpret_cast<const uint16_t*>(rawp + 128 * 64)[r];
-          mbar_arrive(&raw_empty[slot]);
-          const uint32_t s2 = sbits | (sbits << 16);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            deq_int4_word(wv[c].x, s2, &av[16 * c + 0]);
-            deq_int4_word(wv[c].y, s2, &av[16 * c + 4]);
-            deq_int4_word(wv[c].z, s2, &av[16 * c + 8]);
-            deq_int4_word(wv[c].w, s2, &av[16 * c + 12]);
-          }
-        } else {
-          uint4 wv[8];
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            wv[c] = *reinterpret_cast<const uint4*>(rawp + r * 128 + ((c ^ (r & 7)) << 4));
-          mbar_arrive(&raw_empty[slot]);
-          if (fmt == QMOE_W_FP8_E4M3_PC) {
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              deq_fp8_word(wv[c].x, &av[8 * c + 0]);
-              deq_fp8_word(wv[c].y, &av[8 * c + 2]);
-              deq_fp8_word(wv[c].z, &av[8 * c + 4]);
-              deq_fp8_word(wv[c].w, &av[8 * c + 6]);
-            }
-          } else {
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              deq_int8_word(wv[c].x, &av[8 * c + 0]);
-              deq_int8_word(wv[c].y, &av[8 * c + 2]);
-              deq_int8_word(wv[c].z, &av[8 * c + 4]);
-              deq_int8_word(wv[c].w, &av[8 * c + 6]);
-            }
-          }
-        }
-        const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + C::A_COL0 + s * 64;
-        tmem_st16(taddr + 0, &av[0]);
-        tmem_st16(taddr + 16, &av[16]);
-        tmem_st16(taddr + 32, &av[32]);
-        tmem_st16(taddr + 48, &av[48]);
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&full[s]);
-      }
+      for (int c = 0; c < kKW / 32; ++c) tmem_st16(tbase + s * 64 + 16 * c, &av[16 * c]);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&full[s]);
+      if (++s == (uint32_t)C::SA) { s = 0; ph ^= 1; }
+      --left;
     }
-    cp_async_wait_all();
   } else {
     // ---------------- epilogue ----------------
-    // Each warp owns 32 accumulator rows (TMEM lane quarter q) and stages and
-    // stores its own slice of the output rows, so only warp-level syncs are
-    // needed.  mat 0: 16 intermediate columns (32 B) per token;
-    // mat 1: 32 output columns (64 B) per token.
+    // Each of the 4 epilogue warps owns 32 accumulator rows (TMEM lane
+    // quarter q) and stages and stores its own slice of the output rows, so
+    // only warp-level syncs are needed.  mat 0: 16 intermediate columns
+    // (32 B) per token; mat 1: 32 output columns (64 B) per token.
     const int q = warp & 3;
     const int r = 32 * q + lane;             // accumulator row = tile weight row
     constexpr int WCOLS = MAT == 0 ? 16 : 32;
@@ -367,8 +419,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
       const Tile t = decode_tile(tile, tab_off, s_seg_off, s_seg_cnt, n_seg, BN);
       const int b = tc & 1;
       const ExpertDev& ex = a.experts[t.seg];
-      const float scale = ex.spc[MAT] ? ex.spc[MAT][t.mb * 128 + r] : 1.0f;
-      ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[b], (tc >> 1) & 1, abort_flag));
+      const float scale = (FMT != QMOE_W_INT4_G128) ? ex.spc[MAT][t.mb * 128 + r] : 1.0f;
+      ok = warp_wait(&acc_full[b], (tc >> 1) & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
       const int n_mma = max(16, (t.nvalid + 15) & ~15);
@@ -390,8 +442,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
         }
       }
       tc_fence_before();
-      mbar_arrive(&acc_empty[b]);
       __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[b]);
       constexpr int VPR = WCOLS / 8;         // 16-byte vectors per token row slice
       const int col0 = MAT == 0 ? t.mb * 64 + q * 16 : t.mb * 128 + q * 32;
       for (int v = lane; v < t.nvalid * VPR; v += 32) {
@@ -405,33 +457,49 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == kRawWarp) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }
   if (tid == 0 && *abort_flag) atomicOr(a.err, kErrTimeout);
 }
 
-template <int BN>
-cudaError_t launch_bn(const GemmArgs& a, int num_sms, cudaStream_t s) {
-  using C = Cfg<BN>;
-  auto kern = a.mat == 0 ? grouped_gemm_kernel<BN, 0> : grouped_gemm_kernel<BN, 1>;
+template <int BN, int MAT, int FMT>
+cudaError_t launch_one(const GemmArgs& a, const CUtensorMap& map, int num_sms, cudaStream_t s) {
+  using C = Cfg<BN, FMT>;
+  auto kern = grouped_gemm_kernel<BN, MAT, FMT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<num_sms, kThreads, C::SMEM, s>>>(a);
+  kern<<<num_sms, kThreads, C::SMEM, s>>>(a, map);
   return cudaGetLastError();
+}
+
+template <int BN, int MAT>
+cudaError_t launch_fmt(const GemmArgs& a, const CUtensorMap& map, int fmt, int num_sms, cudaStream_t s) {
+  switch (fmt) {
+    case QMOE_W_INT4_G128: return launch_one<BN, MAT, QMOE_W_INT4_G128>(a, map, num_sms, s);
+    case QMOE_W_FP8_E4M3_PC: return launch_one<BN, MAT, QMOE_W_FP8_E4M3_PC>(a, map, num_sms, s);
+    case QMOE_W_INT8_PC: return launch_one<BN, MAT, QMOE_W_INT8_PC>(a, map, num_sms, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int BN>
+cudaError_t launch_bn(const GemmArgs& a, const CUtensorMap& map, int fmt, int num_sms, cudaStream_t s) {
+  return a.mat == 0 ? launch_fmt<BN, 0>(a, map, fmt, num_sms, s) : launch_fmt<BN, 1>(a, map, fmt, num_sms, s);
 }
 
 }  // namespace
 
 bool gemm_bn_supported(int bn) { return bn == 16 || bn == 32 || bn == 64 || bn == 128; }
 
-cudaError_t launch_grouped_gemm(const GemmArgs& a, int bn, int num_sms, cudaStream_t s) {
+cudaError_t launch_grouped_gemm(const GemmArgs& a, const CUtensorMap& act_map, int fmt, int bn, int num_sms,
+                                cudaStream_t s) {
   switch (bn) {
-    case 16: return launch_bn<16>(a, num_sms, s);
-    case 32: return launch_bn<32>(a, num_sms, s);
-    case 64: return launch_bn<64>(a, num_sms, s);
-    case 128: return launch_bn<128>(a, num_sms, s);
+    case 16: return launch_bn<16>(a, act_map, fmt, num_sms, s);
+    case 32: return launch_bn<32>(a, act_map, fmt, num_sms, s);
+    case 64: return launch_bn<64>(a, act_map, fmt, num_sms, s);
+    case 128: return launch_bn<128>(a, act_map, fmt, num_sms, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
+#include <cuda.h>
 
 #include "../../include/qmoe.h"
 
@@ -88,23 +89,40 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
   return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity.  Gives up (returns
-// false) when *abort is raised by another role or after ~2^31 SM cycles
-// (about a second), in which case it raises *abort itself.
+// try_wait with a suspend-time hint: the warp sleeps in hardware until the
+// phase completes or about 10 ms pass, so waiting roles take no issue slots.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar_addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar_addr), "r"(parity), "r"(10000000u)
+      : "memory");
+  return ok != 0;
+}
+
+// Slow path of mbar_wait: sleep-wait with a bound.  Gives up (returns false)
+// when *abort is raised by another role or after ~2^31 SM cycles (about a
+// second), in which case it raises *abort itself.
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t addr, uint32_t parity, volatile int* abort) {
+  const long long t0 = clock64();
+  for (;;) {
+    if (mbar_try_wait_sleep(addr, parity)) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > (1ll << 31)) {
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+// Bounded wait for the phase with the given parity (fast path inline).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   const uint32_t addr = smem_u32(bar);
   if (mbar_try_wait(addr, parity)) return true;
-  const long long t0 = clock64();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(addr, parity)) return true;
-    if ((i & 255u) == 0) {
-      if (*abort) return false;
-      if (clock64() - t0 > (1ll << 31)) {
-        *abort = 1;
-        return false;
-      }
-    }
-  }
+  return mbar_wait_slow(addr, parity, abort);
 }
 
 // Same, ignoring the abort flag (used while draining on the way out).
@@ -227,20 +245,29 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
 // ---------------------------------------------------------------------------
 // host-side launchers (implemented in the .cu files)
 // ---------------------------------------------------------------------------
-cudaError_t launch_router_logits(const uint16_t* x, const float* Wr, int T, int d, int E, int split,
-                                 float* zpart, cudaStream_t s);
-cudaError_t launch_router_topk(const float* zpart, int split, const float* bias, int T, int E, int k,
-                               int32_t* idx, float* gate, cudaStream_t s);
+cudaError_t launch_router(const uint16_t* x, const float* Wr, const float* bias, int T, int d, int E, int k,
+                          int split, float* zpart, int* tickets, int32_t* idx, float* gate, cudaStream_t s);
+cudaError_t launch_router_topk(const float* logits, int T, int E, int k, int32_t* idx, float* gate, cudaStream_t s);
 int router_split(int T, int d, int E, int num_sms);
+int router_tickets(int max_tokens);
 
-cudaError_t launch_schedule(const int32_t* idx, int T, int k, int E, int S, int bn3, int mb3, int bn4, int mb4,
-                            int32_t* counts, int32_t* offsets, int32_t* sorted_token, int32_t* inv_pos,
-                            int32_t* seg_off, int32_t* seg_cnt, int32_t* tile3_off, int32_t* tile4_off,
-                            int32_t* scratch, cudaStream_t s);
+// Tile tables written by the schedule kernel: for matrix m (0 gate/up, 1
+// down) and weight format f (1..3), tiles + tile_table_offset(m, f, n_seg)
+// holds the n_seg + 1 prefix sums of the tiles of the segments in format f.
+__host__ __device__ inline int tile_table_offset(int mat, int fmt, int n_seg) {
+  return (mat * 3 + (fmt - 1)) * (n_seg + 1);
+}
+
+cudaError_t launch_schedule(const int32_t* idx, int T, int k, int E, int S, int bn, int mb3, int mb4,
+                            const int32_t* seg_fmt, int32_t* counts, int32_t* offsets, int32_t* sorted_token,
+                            int32_t* inv_pos, int32_t* seg_off, int32_t* seg_cnt, int32_t* tiles, int32_t* scratch,
+                            cudaStream_t s);
 size_t schedule_scratch_ints(int max_tokens, int E);
 
-cudaError_t launch_grouped_gemm(const GemmArgs& a, int bn, int num_sms, cudaStream_t s);
 bool gemm_bn_supported(int bn);
+
+cudaError_t launch_grouped_gemm(const GemmArgs& a, const CUtensorMap& act_map, int fmt, int bn, int num_sms,
+                                cudaStream_t s);
 
 cudaError_t launch_combine(const uint16_t* Y, const float* gate, const int32_t* inv_pos, int T, int k, int S,
                            int d, uint16_t* out, cudaStream_t s);

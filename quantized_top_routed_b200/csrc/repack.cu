@@ -8,15 +8,18 @@
 //     2j+1 is the matching up row I + 64*mb + j, so the SwiGLU epilogue
 //     finds gate and up of one intermediate index in neighbouring lanes;
 //   down matrix (mat 1): tile row r is weight row 128*mb + r.
-// Byte order inside a row (chosen for the in-register dequantisation):
-//   INT8 / FP8: each 32-bit word holds K elements (k0, k2, k1, k3) in bytes
-//     0..3, so bytes {0,2} and {1,3} expand to bf16 pairs (k0,k1), (k2,k3);
-//     16-byte chunk c of row r is stored at chunk position c ^ (r & 7).
-//   INT4: each 32-bit word holds 8 K elements as biased nibbles (q + 8);
-//     nibble n < 4 is element 2n, nibble n >= 4 is element 2(n-4)+1, so
-//     (w >> 4j) & 0x000F000F yields the pair (2j, 2j+1); chunk c of row r is
-//     stored at position c ^ ((r >> 1) & 3).  The 128 bf16 group scales of
-//     the tile (one per row) follow the 8192 code bytes.
+// Chunk order: the tile is stored chunk-major, 16-byte chunk c of row r at
+// byte c * 2048 + r * 16, so the 32 rows of a warp read one chunk as 512
+// contiguous bytes (one coalesced 16-byte load per lane).
+// Byte order inside a chunk (chosen for the in-register dequantisation):
+//   INT8 / FP8 (16 K elements per chunk): each 32-bit word holds K elements
+//     (k0, k2, k1, k3) in bytes 0..3, so bytes {0,2} and {1,3} expand to
+//     bf16 pairs (k0,k1), (k2,k3).
+//   INT4 (32 K elements per chunk): each 32-bit word holds 8 K elements as
+//     biased nibbles (q + 8); nibble n < 4 is element 2n, nibble n >= 4 is
+//     element 2(n-4)+1, so (w >> 4j) & 0x000F000F yields the pair (2j, 2j+1).
+//     The 128 bf16 group scales of the tile (one per row) follow the 8192
+//     code bytes.
 // Per-channel scales (INT8 / FP8) are written in tile-row order.
 #include "qmoe_internal.cuh"
 
@@ -55,7 +58,7 @@ __global__ void repack_kernel(int fmt, int mat, const uint8_t* __restrict__ w, c
         }
         words[m] = v;
       }
-      uint4* o = reinterpret_cast<uint4*>(tile + r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
+      uint4* o = reinterpret_cast<uint4*>(tile + c * 2048 + r * 16);
       *o = make_uint4(words[0], words[1], words[2], words[3]);
     }
     const uint16_t* sc = static_cast<const uint16_t*>(scale);
@@ -68,7 +71,7 @@ __global__ void repack_kernel(int fmt, int mat, const uint8_t* __restrict__ w, c
         const uint8_t* p = s + 16 * c + 4 * m;
         words[m] = (uint32_t)p[0] | ((uint32_t)p[2] << 8) | ((uint32_t)p[1] << 16) | ((uint32_t)p[3] << 24);
       }
-      uint4* o = reinterpret_cast<uint4*>(tile + r * 128 + ((c ^ (r & 7)) << 4));
+      uint4* o = reinterpret_cast<uint4*>(tile + c * 2048 + r * 16);
       *o = make_uint4(words[0], words[1], words[2], words[3]);
     }
     if (ks == 0) dst_spc[rg] = static_cast<const float*>(scale)[src];

@@ -5,13 +5,14 @@
 // top-k routing; "FineRMoE", Sparse Sum Layer: softmax probabilities as
 // mixing weights.)
 //
-// Two kernels:
-//  * router_logits_kernel: a 32-token x 32-expert fp32 tile per CTA over one
-//    slice of d (d is split so the grid covers the SMs when T is small).
-//    Each slice's partial sums go to zpart[slice][T][E]; the summation order
-//    is fixed, so the logits are deterministic.
-//  * router_topk_kernel: one warp per token; the E logits live in registers
-//    (ceil(E/32) per lane), top-k is k rounds of a warp arg-max.
+// From activations (one launch): router_fused_kernel computes a 32-token x
+// 32-expert tile of fp32 logits over one slice of d (d is split so the grid
+// covers the SMs when T is small), streaming x and Wr through a 3-stage
+// cp.async ring.  Each CTA writes its partial sums, then takes a ticket for
+// its token tile; the CTA that completes the tile sums the partials of all
+// slices in a fixed order (so the logits are deterministic) and runs the
+// warp-per-token top-k for the tile's 32 tokens, then resets the ticket.
+// From supplied logits: router_topk_kernel alone, one warp per token.
 #include "qmoe_internal.cuh"
 
 #include <math.h>
@@ -19,63 +20,15 @@
 namespace qmoe {
 namespace {
 
-constexpr int RT = 32;   // tokens per CTA
-constexpr int RE = 32;   // experts per CTA
-constexpr int RC = 32;   // d elements per smem chunk
-constexpr int RS = RC + 4;
-
-__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
-
-__global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __restrict__ x,
-                                                            const float* __restrict__ Wr, int T, int d,
-                                                            int E, int slice, float* __restrict__ zpart) {
-  __shared__ __align__(16) float xs[RT][RS];
-  __shared__ __align__(16) float ws[RE][RS];
-  const int t0 = blockIdx.x * RT, e0 = blockIdx.y * RE, c_begin = blockIdx.z * slice;
-  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-  const int lr = tid >> 3, lc = (tid & 7) * 4;   // loader: row, column
-  float acc00 = 0.f, acc01 = 0.f, acc10 = 0.f, acc11 = 0.f;  // [token ty|ty+16][expert tx|tx+16]
-
-  for (int c0 = c_begin; c0 < c_begin + slice; c0 += RC) {
-    {
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      const int t = t0 + lr;
-      if (t < T) {
-        const uint2 raw = *reinterpret_cast<const uint2*>(x + (size_t)t * d + c0 + lc);
-        v = make_float4(bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y));
-      }
-      *reinterpret_cast<float4*>(&xs[lr][lc]) = v;
-      float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
-      const int e = e0 + lr;
-      if (e < E) w = *reinterpret_cast<const float4*>(Wr + (size_t)e * d + c0 + lc);
-      *reinterpret_cast<float4*>(&ws[lr][lc]) = w;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int c = 0; c < RC; c += 4) {
-      const float4 a0 = *reinterpret_cast<const float4*>(&xs[ty][c]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&xs[ty + 16][c]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&ws[tx][c]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&ws[tx + 16][c]);
-      acc00 = fmaf(a0.x, b0.x, acc00); acc00 = fmaf(a0.y, b0.y, acc00);
-      acc00 = fmaf(a0.z, b0.z, acc00); acc00 = fmaf(a0.w, b0.w, acc00);
-      acc01 = fmaf(a0.x, b1.x, acc01); acc01 = fmaf(a0.y, b1.y, acc01);
-      acc01 = fmaf(a0.z, b1.z, acc01); acc01 = fmaf(a0.w, b1.w, acc01);
-      acc10 = fmaf(a1.x, b0.x, acc10); acc10 = fmaf(a1.y, b0.y, acc10);
-      acc10 = fmaf(a1.z, b0.z, acc10); acc10 = fmaf(a1.w, b0.w, acc10);
-      acc11 = fmaf(a1.x, b1.x, acc11); acc11 = fmaf(a1.y, b1.y, acc11);
-      acc11 = fmaf(a1.z, b1.z, acc11); acc11 = fmaf(a1.w, b1.w, acc11);
-    }
-    __syncthreads();
-  }
-  float* zp = zpart + (size_t)blockIdx.z * T * E;
-  const int ta = t0 + ty, tb = t0 + ty + 16, ea = e0 + tx, eb = e0 + tx + 16;
-  if (ta < T && ea < E) zp[(size_t)ta * E + ea] = acc00;
-  if (ta < T && eb < E) zp[(size_t)ta * E + eb] = acc01;
-  if (tb < T && ea < E) zp[(size_t)tb * E + ea] = acc10;
-  if (tb < T && eb < E) zp[(size_t)tb * E + eb] = acc11;
-}
+constexpr int RT = 32;          // tokens per CTA
+constexpr int RE = 32;          // experts per CTA
+constexpr int RC = 128;         // d elements per pipeline stage
+constexpr int NST = 3;          // cp.async stages
+constexpr int XS = RC + 8;      // bf16 row stride of the x stage (bank shift of 4 words per row)
+constexpr int WS = RC + 4;      // fp32 row stride of the Wr stage
+constexpr int kRouterThreads = 256;
+constexpr int kSmemPipe = NST * (RT * XS * 2 + RE * WS * 4);
+constexpr int kSmemRouter = kSmemPipe > RT * kMaxE * 4 ? kSmemPipe : RT * kMaxE * 4;
 
 // Warp arg-max over (value, index): larger value wins, lower index on ties.
 __device__ __forceinline__ void warp_argmax(float& v, int& e) {
@@ -90,13 +43,11 @@ __device__ __forceinline__ void warp_argmax(float& v, int& e) {
   }
 }
 
-template <int EPL>
-__global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ zpart, int split,
-                                                          const float* __restrict__ bias, int T, int E, int k,
-                                                          int32_t* __restrict__ idx, float* __restrict__ gate) {
-  const int t = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
-  const int lane = threadIdx.x & 31;
-  if (t >= T) return;
+// One warp: softmax + top-k + renormalisation of one token's E logits.
+// logit(e) gives the fp32 logit of expert e (bias included).
+template <int EPL, class LogitFn>
+__device__ __forceinline__ void topk_token(LogitFn logit, int E, int k, int lane, int32_t* idx_row,
+                                           float* gate_row) {
   float z[EPL];
   bool live[EPL];
   float m = -INFINITY;
@@ -104,14 +55,8 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
   for (int i = 0; i < EPL; ++i) {
     const int e = lane + 32 * i;
     live[i] = e < E;
-    float v = -INFINITY;
-    if (live[i]) {
-      v = 0.f;
-      for (int s = 0; s < split; ++s) v += zpart[((size_t)s * T + t) * E + e];
-      if (bias) v += bias[e];
-    }
-    z[i] = v;
-    m = fmaxf(m, v);
+    z[i] = live[i] ? logit(e) : -INFINITY;
+    m = fmaxf(m, z[i]);
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
@@ -122,7 +67,6 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
 
-  // k rounds of arg-max; lane j keeps slot j.
   float my_p = 0.f;
   int my_e = 0;
   for (int j = 0; j < k; ++j) {
@@ -149,9 +93,141 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, off);
   if (lane < k) {
-    idx[(size_t)t * k + lane] = my_e;
-    gate[(size_t)t * k + lane] = my_p / psum;
+    idx_row[lane] = my_e;
+    gate_row[lane] = my_p / psum;
   }
+}
+
+__device__ __forceinline__ void cp16(uint32_t dst, const void* src, uint32_t n) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
+}
+
+template <int EPL>
+__global__ void __launch_bounds__(kRouterThreads) router_fused_kernel(
+    const uint16_t* __restrict__ x, const float* __restrict__ Wr, const float* __restrict__ bias, int T, int d,
+    int E, int k, int split, float* __restrict__ zpart, int* __restrict__ tickets, int32_t* __restrict__ idx,
+    float* __restrict__ gate) {
+  extern __shared__ __align__(16) uint8_t rsm[];
+  uint16_t* xs = reinterpret_cast<uint16_t*>(rsm);                          // [NST][RT][XS]
+  float* ws = reinterpret_cast<float*>(rsm + NST * RT * XS * 2);            // [NST][RE][WS]
+  __shared__ int s_last;
+  const int tt = blockIdx.x, et = blockIdx.y, sp = blockIdx.z;
+  const int t0 = tt * RT, e0 = et * RE;
+  const int slice = d / split, c_begin = sp * slice, nchunks = slice / RC;
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+
+  auto issue = [&](int chunk, int stage) {
+    const int c0 = c_begin + chunk * RC;
+    const uint32_t xb = smem_u32(xs + stage * RT * XS);
+    const uint32_t wb = smem_u32(ws + stage * RE * WS);
+#pragma unroll
+    for (int i = 0; i < (RT * RC * 2 / 16) / kRouterThreads; ++i) {  // x: 16 chunks of 16 B per row
+      const int v = tid + i * kRouterThreads, row = v >> 4, c = v & 15;
+      const int t = t0 + row;
+      cp16(xb + (row * XS + c * 8) * 2, x + (size_t)min(t, T - 1) * d + c0 + c * 8, t < T ? 16 : 0);
+    }
+#pragma unroll
+    for (int i = 0; i < (RE * RC * 4 / 16) / kRouterThreads; ++i) {  // Wr: 32 chunks of 16 B per row
+      const int v = tid + i * kRouterThreads, row = v >> 5, c = v & 31;
+      const int e = e0 + row;
+      cp16(wb + (row * WS + c * 4) * 4, Wr + (size_t)min(e, E - 1) * d + c0 + c * 4, e < E ? 16 : 0);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+
+  float acc00 = 0.f, acc01 = 0.f, acc10 = 0.f, acc11 = 0.f;  // [token ty|ty+16][expert tx|tx+16]
+#pragma unroll
+  for (int p = 0; p < NST - 1; ++p)
+    if (p < nchunks) issue(p, p);
+    else asm volatile("cp.async.commit_group;" ::: "memory");
+  for (int c = 0; c < nchunks; ++c) {
+    asm volatile("cp.async.wait_group %0;" ::"n"(NST - 2) : "memory");
+    __syncthreads();
+    if (c + NST - 1 < nchunks) issue(c + NST - 1, (c + NST - 1) % NST);
+    else asm volatile("cp.async.commit_group;" ::: "memory");
+    const uint16_t* xa = xs + (c % NST) * RT * XS + ty * XS;
+    const uint16_t* xb = xa + 16 * XS;
+    const float* wa = ws + (c % NST) * RE * WS + tx * WS;
+    const float* wb = wa + 16 * WS;
+#pragma unroll 8
+    for (int i = 0; i < RC; i += 4) {
+      const uint2 ua = *reinterpret_cast<const uint2*>(xa + i);
+      const uint2 ub = *reinterpret_cast<const uint2*>(xb + i);
+      const float4 va = *reinterpret_cast<const float4*>(wa + i);
+      const float4 vb = *reinterpret_cast<const float4*>(wb + i);
+      const float a0 = __uint_as_float(ua.x << 16), a1 = __uint_as_float(ua.x & 0xFFFF0000u);
+      const float a2 = __uint_as_float(ua.y << 16), a3 = __uint_as_float(ua.y & 0xFFFF0000u);
+      const float b0 = __uint_as_float(ub.x << 16), b1 = __uint_as_float(ub.x & 0xFFFF0000u);
+      const float b2 = __uint_as_float(ub.y << 16), b3 = __uint_as_float(ub.y & 0xFFFF0000u);
+      acc00 = fmaf(a0, va.x, acc00); acc00 = fmaf(a1, va.y, acc00);
+      acc00 = fmaf(a2, va.z, acc00); acc00 = fmaf(a3, va.w, acc00);
+      acc01 = fmaf(a0, vb.x, acc01); acc01 = fmaf(a1, vb.y, acc01);
+      acc01 = fmaf(a2, vb.z, acc01); acc01 = fmaf(a3, vb.w, acc01);
+      acc10 = fmaf(b0, va.x, acc10); acc10 = fmaf(b1, va.y, acc10);
+      acc10 = fmaf(b2, va.z, acc10); acc10 = fmaf(b3, va.w, acc10);
+      acc11 = fmaf(b0, vb.x, acc11); acc11 = fmaf(b1, vb.y, acc11);
+      acc11 = fmaf(b2, vb.z, acc11); acc11 = fmaf(b3, vb.w, acc11);
+    }
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+
+  float* zp = zpart + (size_t)sp * T * E;
+  const int ta = t0 + ty, tb = t0 + ty + 16, ea = e0 + tx, eb = e0 + tx + 16;
+  if (ta < T && ea < E) zp[(size_t)ta * E + ea] = acc00;
+  if (ta < T && eb < E) zp[(size_t)ta * E + eb] = acc01;
+  if (tb < T && ea < E) zp[(size_t)tb * E + ea] = acc10;
+  if (tb < T && eb < E) zp[(size_t)tb * E + eb] = acc11;
+
+  // ---- the CTA that completes a token tile runs its top-k ----------------
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const int need = gridDim.y * gridDim.z;
+    const int ticket = atomicAdd(&tickets[tt], 1);
+    s_last = ticket == need - 1;
+    if (s_last) tickets[tt] = 0;  // ready for the next call
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // Sum the slices of this tile's logits into shared memory (coalesced,
+  // every load in flight at once), then one warp per token runs the top-k.
+  float* zs = reinterpret_cast<float*>(rsm);                   // [RT][E], reuses the pipeline buffers
+  const int rows = min(RT, T - t0);
+  for (int v = tid; v < rows * E; v += kRouterThreads) {
+    const int r = v / E, e = v - r * E;
+    float acc = 0.f;
+    for (int s2 = 0; s2 < split; ++s2) acc += __ldcg(zpart + ((size_t)s2 * T + t0 + r) * E + e);
+    zs[v] = bias ? acc + bias[e] : acc;
+  }
+  __syncthreads();
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int r = warp; r < rows; r += kRouterThreads / 32) {
+    const int t = t0 + r;
+    auto logit = [&](int e) { return zs[r * E + e]; };
+    topk_token<EPL>(logit, E, k, lane, idx + (size_t)t * k, gate + (size_t)t * k);
+  }
+}
+
+template <int EPL>
+__global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                          int32_t* __restrict__ idx, float* __restrict__ gate) {
+  const int t = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  auto logit = [&](int e) { return logits[(size_t)t * E + e]; };
+  topk_token<EPL>(logit, E, k, lane, idx + (size_t)t * k, gate + (size_t)t * k);
+}
+
+template <int EPL>
+cudaError_t launch_fused(const uint16_t* x, const float* Wr, const float* bias, int T, int d, int E, int k, int split,
+                         float* zpart, int* tickets, int32_t* idx, float* gate, cudaStream_t s) {
+  auto kern = router_fused_kernel<EPL>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemRouter);
+  if (e != cudaSuccess) return e;
+  dim3 grid((T + RT - 1) / RT, (E + RE - 1) / RE, split);
+  kern<<<grid, kRouterThreads, kSmemRouter, s>>>(x, Wr, bias, T, d, E, k, split, zpart, tickets, idx, gate);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -159,29 +235,35 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
 int router_split(int T, int d, int E, int num_sms) {
   const int tiles = ((T + RT - 1) / RT) * ((E + RE - 1) / RE);
   int split = 1;
-  // split d while the grid is short of the SM count and slices stay >= 256
-  while (tiles * split * 2 <= num_sms && d % (split * 2 * RC) == 0 && d / (split * 2) >= 256 && split < 16)
+  // split d while the grid is short of the SM count and every slice keeps >= 2 stages
+  while (tiles * split * 2 <= num_sms && d % (split * 2 * RC) == 0 && d / (split * 2) >= 2 * RC && split < 16)
     split *= 2;
   return split;
 }
 
-cudaError_t launch_router_logits(const uint16_t* x, const float* Wr, int T, int d, int E, int split, float* zpart,
-                                 cudaStream_t s) {
-  dim3 grid((T + RT - 1) / RT, (E + RE - 1) / RE, split);
-  router_logits_kernel<<<grid, 256, 0, s>>>(x, Wr, T, d, E, d / split, zpart);
-  return cudaGetLastError();
+int router_tickets(int max_tokens) { return (max_tokens + RT - 1) / RT; }
+
+cudaError_t launch_router(const uint16_t* x, const float* Wr, const float* bias, int T, int d, int E, int k, int split,
+                          float* zpart, int* tickets, int32_t* idx, float* gate, cudaStream_t s) {
+  const int epl = (E + 31) / 32;
+  switch (epl) {
+    case 1: return launch_fused<1>(x, Wr, bias, T, d, E, k, split, zpart, tickets, idx, gate, s);
+    case 2: return launch_fused<2>(x, Wr, bias, T, d, E, k, split, zpart, tickets, idx, gate, s);
+    case 3:
+    case 4: return launch_fused<4>(x, Wr, bias, T, d, E, k, split, zpart, tickets, idx, gate, s);
+    default: return launch_fused<8>(x, Wr, bias, T, d, E, k, split, zpart, tickets, idx, gate, s);
+  }
 }
 
-cudaError_t launch_router_topk(const float* zpart, int split, const float* bias, int T, int E, int k, int32_t* idx,
-                               float* gate, cudaStream_t s) {
+cudaError_t launch_router_topk(const float* logits, int T, int E, int k, int32_t* idx, float* gate, cudaStream_t s) {
   const int blocks = (T + 7) / 8;
   const int epl = (E + 31) / 32;
   switch (epl) {
-    case 1: router_topk_kernel<1><<<blocks, 256, 0, s>>>(zpart, split, bias, T, E, k, idx, gate); break;
-    case 2: router_topk_kernel<2><<<blocks, 256, 0, s>>>(zpart, split, bias, T, E, k, idx, gate); break;
+    case 1: router_topk_kernel<1><<<blocks, 256, 0, s>>>(logits, T, E, k, idx, gate); break;
+    case 2: router_topk_kernel<2><<<blocks, 256, 0, s>>>(logits, T, E, k, idx, gate); break;
     case 3:
-    case 4: router_topk_kernel<4><<<blocks, 256, 0, s>>>(zpart, split, bias, T, E, k, idx, gate); break;
-    default: router_topk_kernel<8><<<blocks, 256, 0, s>>>(zpart, split, bias, T, E, k, idx, gate); break;
+    case 4: router_topk_kernel<4><<<blocks, 256, 0, s>>>(logits, T, E, k, idx, gate); break;
+    default: router_topk_kernel<8><<<blocks, 256, 0, s>>>(logits, T, E, k, idx, gate); break;
   }
   return cudaGetLastError();
 }

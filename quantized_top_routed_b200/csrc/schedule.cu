@@ -21,6 +21,7 @@ namespace qmoe {
 namespace {
 
 constexpr int kThreads = 1024;
+constexpr size_t kHistSmemMax = 160 * 1024;   // dynamic shared memory for chunk histograms
 
 __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
 #pragma unroll
@@ -32,14 +33,16 @@ __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    schedule_kernel(const int32_t* __restrict__ idx, int T, int k, int E, int S, int bn3, int mb3, int bn4,
-                    int mb4, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+    schedule_kernel(const int32_t* __restrict__ idx, int T, int k, int E, int S, int bn, int mb3, int mb4,
+                    const int32_t* __restrict__ seg_fmt, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                     int32_t* __restrict__ sorted_token, int32_t* __restrict__ inv_pos,
-                    int32_t* __restrict__ seg_off, int32_t* __restrict__ seg_cnt, int32_t* __restrict__ tile3_off,
-                    int32_t* __restrict__ tile4_off, int32_t* __restrict__ hist) {
+                    int32_t* __restrict__ seg_off, int32_t* __restrict__ seg_cnt, int32_t* __restrict__ tiles,
+                    int32_t* __restrict__ hist_global, int hist_in_smem) {
+  extern __shared__ int32_t hist_smem[];
   __shared__ uint32_t bal[32][kMaxE];
   __shared__ int32_t s_cnt[kMaxE + kMaxShared];
   __shared__ int32_t s_off[kMaxE + 1];
+  int32_t* hist = hist_in_smem ? hist_smem : hist_global;   // [C][E]: chunk counts, then chunk bases
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int C = (T + 31) / 32;
   const uint32_t lt_mask = (1u << lane) - 1u;
@@ -48,13 +51,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int c = warp; c < C; c += 32) {
     const int t = c * 32 + lane;
     const bool valid = t < T;
+    int my[kMaxK];
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) my[j] = (valid && j < k) ? idx[(size_t)t * k + j] : -1;
     for (int w0 = 0; w0 < E; w0 += 32) {
       uint32_t m = 0;
-      if (valid)
-        for (int j = 0; j < k; ++j) {
-          const int e = idx[(size_t)t * k + j] - w0;
-          if (e >= 0 && e < 32) m |= 1u << e;
-        }
+#pragma unroll
+      for (int j = 0; j < kMaxK; ++j) {
+        const int e = my[j] - w0;
+        if (e >= 0 && e < 32) m |= 1u << e;
+      }
       uint32_t mine = 0;
 #pragma unroll 8
       for (int b = 0; b < 32; ++b) {
@@ -63,15 +69,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (w0 + lane < E) {
         bal[warp][w0 + lane] = mine;
-        hist[(size_t)c * E + w0 + lane] = __popc(mine);
+        hist[c * E + w0 + lane] = __popc(mine);
       }
     }
     __syncwarp();
-    if (valid)
-      for (int j = 0; j < k; ++j) {
-        const int e = idx[(size_t)t * k + j];
-        inv_pos[(size_t)t * k + j] = __popc(bal[warp][e] & lt_mask);  // rank for now
-      }
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+      if (my[j] >= 0) inv_pos[(size_t)t * k + j] = __popc(bal[warp][my[j]] & lt_mask);  // rank for now
     __syncwarp();
   }
   __syncthreads();
@@ -81,12 +85,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int per = (C + 31) / 32;
     const int c0 = min(C, lane * per), c1 = min(C, c0 + per);
     int sum = 0;
-    for (int c = c0; c < c1; ++c) sum += hist[(size_t)c * E + e];
+    for (int c = c0; c < c1; ++c) sum += hist[c * E + e];
     const int incl = warp_incl_scan(sum, lane);
     int run = incl - sum;
     for (int c = c0; c < c1; ++c) {
-      const int h = hist[(size_t)c * E + e];
-      hist[(size_t)c * E + e] = run;
+      const int h = hist[c * E + e];
+      hist[c * E + e] = run;
       run += h;
     }
     if (lane == 31) s_cnt[e] = incl;
@@ -109,7 +113,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int p = tid; p < P; p += kThreads) {
     const int t = p / k;
     const int e = idx[p];
-    const int pos = s_off[e] + hist[(size_t)(t >> 5) * E + e] + inv_pos[p];
+    const int pos = s_off[e] + hist[(t >> 5) * E + e] + inv_pos[p];
     sorted_token[pos] = t;
     inv_pos[p] = pos;
   }
@@ -118,37 +122,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int p = tid; p < S * T; p += kThreads) sorted_token[P + p] = p % T;
 
   // ---- segment and tile tables for the grouped GEMMs ------------------------
+  // One prefix-sum table per (matrix, weight format): segments of another
+  // format contribute no tiles, so each per-format launch walks only its own.
   if (seg_off == nullptr) return;
   const int n_seg = E + S;
-  if (warp == 0) {
-    int run3 = 0, run4 = 0;
+  for (int e = tid; e < n_seg; e += kThreads) {
+    seg_off[e] = e < E ? s_off[e] : P + (e - E) * T;
+    seg_cnt[e] = e < E ? s_cnt[e] : T;
+  }
+  if (warp < 6) {                       // warp w: matrix w / 3, format w % 3 + 1
+    const int mat = warp / 3, fmt = warp % 3 + 1;
+    const int mb = mat == 0 ? mb3 : mb4;
+    int32_t* tab = tiles + tile_table_offset(mat, fmt, n_seg);
+    int run = 0;
     for (int e0 = 0; e0 < n_seg; e0 += 32) {
       const int e = e0 + lane;
-      int cnt = 0, off = 0;
-      if (e < E) {
-        cnt = s_cnt[e];
-        off = s_off[e];
-      } else if (e < n_seg) {
-        cnt = T;
-        off = P + (e - E) * T;
+      int t = 0;
+      if (e < n_seg && seg_fmt[e] == fmt) {
+        const int cnt = e < E ? s_cnt[e] : T;
+        t = ((cnt + bn - 1) / bn) * mb;
       }
-      const int t3 = ((cnt + bn3 - 1) / bn3) * mb3;
-      const int t4 = ((cnt + bn4 - 1) / bn4) * mb4;
-      const int i3 = warp_incl_scan(t3, lane);
-      const int i4 = warp_incl_scan(t4, lane);
-      if (e < n_seg) {
-        seg_off[e] = off;
-        seg_cnt[e] = cnt;
-        tile3_off[e] = run3 + i3 - t3;
-        tile4_off[e] = run4 + i4 - t4;
-      }
-      run3 += __shfl_sync(0xffffffffu, i3, 31);
-      run4 += __shfl_sync(0xffffffffu, i4, 31);
+      const int incl = warp_incl_scan(t, lane);
+      if (e < n_seg) tab[e] = run + incl - t;
+      run += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) {
-      tile3_off[n_seg] = run3;
-      tile4_off[n_seg] = run4;
-    }
+    if (lane == 0) tab[n_seg] = run;
   }
 }
 
@@ -156,12 +154,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 size_t schedule_scratch_ints(int max_tokens, int E) { return (size_t)((max_tokens + 31) / 32) * E; }
 
-cudaError_t launch_schedule(const int32_t* idx, int T, int k, int E, int S, int bn3, int mb3, int bn4, int mb4,
-                            int32_t* counts, int32_t* offsets, int32_t* sorted_token, int32_t* inv_pos,
-                            int32_t* seg_off, int32_t* seg_cnt, int32_t* tile3_off, int32_t* tile4_off,
-                            int32_t* scratch, cudaStream_t s) {
-  schedule_kernel<<<1, kThreads, 0, s>>>(idx, T, k, E, S, bn3, mb3, bn4, mb4, counts, offsets, sorted_token, inv_pos,
-                                         seg_off, seg_cnt, tile3_off, tile4_off, scratch);
+cudaError_t launch_schedule(const int32_t* idx, int T, int k, int E, int S, int bn, int mb3, int mb4,
+                            const int32_t* seg_fmt, int32_t* counts, int32_t* offsets, int32_t* sorted_token,
+                            int32_t* inv_pos, int32_t* seg_off, int32_t* seg_cnt, int32_t* tiles, int32_t* scratch,
+                            cudaStream_t s) {
+  // chunk histograms live in shared memory when they fit next to the static arrays
+  const size_t hist_bytes = (size_t)((T + 31) / 32) * E * sizeof(int32_t);
+  const int in_smem = hist_bytes <= kHistSmemMax;
+  const size_t dyn = in_smem ? hist_bytes : 0;
+  if (in_smem) {
+    cudaError_t e = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kHistSmemMax);
+    if (e != cudaSuccess) return e;
+  }
+  schedule_kernel<<<1, kThreads, dyn, s>>>(idx, T, k, E, S, bn, mb3, mb4, seg_fmt, counts, offsets, sorted_token,
+                                           inv_pos, seg_off, seg_cnt, tiles, scratch, in_smem);
   return cudaGetLastError();
 }
 

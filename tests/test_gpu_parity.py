@@ -24,7 +24,14 @@ pytestmark = pytest.mark.gpu
 
 REL_L2 = 1e-2
 MAX_ABS = 3e-2
-GATE_TOL = 1e-6
+GATE_TOL = 1e-6      # gates from supplied logits: same fp32 inputs, softmax rounding only
+# Gates from raw x inherit the fp32 rounding of the logits.  A d-term fp32
+# dot product of x ~ N(0,1) with w ~ N(0,1/d) accumulates about
+# 2^-24 * d / sqrt(2) * rms(x_i w_i) ~ 3e-6 of error at d = 4096 (one sigma);
+# the renormalised softmax has |dg/dz| <= 1/2, so gates agree within 1e-5
+# with a wide margin.  The same bound keeps every token with a logit margin
+# above 1e-4 on the oracle's experts.
+GATE_TOL_X = 1e-5
 MARGIN = 1e-4
 
 
@@ -79,7 +86,8 @@ def check_route_from_x(dl, T):
     ref = O.route(L)
     safe = O.margin_safe(ref["margin"], MARGIN)
     np.testing.assert_array_equal(g["idx"][safe], ref["idx"][safe])
-    np.testing.assert_allclose(g["gates"][safe], ref["gates"][safe], rtol=0, atol=GATE_TOL)
+    np.testing.assert_allclose(g["gates"][safe], ref["gates"][safe], rtol=0, atol=GATE_TOL_X)
+    np.testing.assert_allclose(g["gates"].sum(axis=1), 1.0, rtol=0, atol=GATE_TOL)
     assert_schedule_equal(g, O.schedule(g["idx"], L.E))
     return g, int((~safe).sum())
 
@@ -121,6 +129,7 @@ def test_route_from_logits_bit_exact(E, k, T):
     ref = O.route(L, logits=logits)
     np.testing.assert_array_equal(g["idx"], ref["idx"])
     np.testing.assert_allclose(g["gates"], ref["gates"], rtol=0, atol=GATE_TOL)
+    np.testing.assert_allclose(g["gates"].sum(axis=1), 1.0, rtol=0, atol=GATE_TOL)
     assert_schedule_equal(g, ref)
     dl.close()
 
