@@ -59,19 +59,22 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Row-major bf16 matrix [rows][cols] read in 4-row x 64-column gathers into
-// 128-byte-swizzled shared memory.
-bool encode_rows_map(CUtensorMap* m, const void* base, int rows, int cols) {
+// Row-major bf16 matrix [rows][cols] read in boxes of 64 columns x box_rows
+// rows into 128-byte-swizzled shared memory (rows past the end read as zero).
+bool encode_rows_map(CUtensorMap* m, const void* base, int rows, int cols, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  const cuuint32_t box[2] = {64, 1};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+constexpr int kNumBn = 4;                 // token-block widths 16, 32, 64, 128
+int bn_index(int bn) { return bn == 16 ? 0 : bn == 32 ? 1 : bn == 64 ? 2 : 3; }
 
 }  // namespace
 
@@ -87,10 +90,11 @@ struct qmoe_handle {
   int32_t *idx = nullptr, *inv_pos = nullptr, *counts = nullptr, *offsets = nullptr, *sorted_token = nullptr;
   int32_t *seg_off = nullptr, *seg_cnt = nullptr, *tiles = nullptr, *seg_fmt = nullptr, *sched_scratch = nullptr;
   bool fmt_present[4] = {false, false, false, false};
-  CUtensorMap h_map;                     // H rows for the down GEMM's gathers
+  CUtensorMap xp_map[kNumBn];            // permuted x rows (gate/up B operand), one per block width
+  CUtensorMap h_map[kNumBn];             // H rows (down B operand), one per block width
   float *gates = nullptr, *zpart = nullptr;
   int* tickets = nullptr;
-  uint16_t *H = nullptr, *Y = nullptr, *x_stage = nullptr, *out_stage = nullptr;
+  uint16_t *Xp = nullptr, *H = nullptr, *Y = nullptr, *x_stage = nullptr, *out_stage = nullptr;
   int* err = nullptr;
   int zpart_split_max = 1;
   // profiling
@@ -321,9 +325,13 @@ qmoe_status qmoe_create(const qmoe_config* cfg, const float* router_w, const flo
     return bail(st);
   if ((st = h->alloc(&h->zpart, (size_t)h->zpart_split_max * Tm * c.E, "router partials")) != QMOE_OK)
     return bail(st);
+  if ((st = h->alloc(&h->Xp, P * c.d, "permuted x")) != QMOE_OK) return bail(st);
   if ((st = h->alloc(&h->H, P * c.I, "H")) != QMOE_OK) return bail(st);
-  if (!encode_rows_map(&h->h_map, h->H, (int)P, c.I))
-    return bail(fail(QMOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the H buffer"));
+  for (int b = 0; b < kNumBn; ++b) {
+    if (!encode_rows_map(&h->xp_map[b], h->Xp, (int)P, c.d, 16 << b) ||
+        !encode_rows_map(&h->h_map[b], h->H, (int)P, c.I, 16 << b))
+      return bail(fail(QMOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for the activation buffers"));
+  }
   if ((st = h->alloc(&h->Y, P * c.d, "Y")) != QMOE_OK) return bail(st);
   if ((st = h->alloc(&h->x_stage, Tm * c.d, "x staging")) != QMOE_OK) return bail(st);
   if ((st = h->alloc(&h->out_stage, Tm * c.d, "out staging")) != QMOE_OK) return bail(st);
@@ -365,8 +373,7 @@ qmoe_status qmoe_forward(qmoe_handle* h, const uint16_t* x, int32_t T, uint16_t*
   st = route_impl(h, x, nullptr, T, h->idx, h->gates, h->counts, h->offsets, h->sorted_token, h->inv_pos, true, bn, s);
   if (st != QMOE_OK) return st;
 
-  CUtensorMap x_map;
-  if (!encode_rows_map(&x_map, x, T, c.d)) return fail(QMOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for x");
+  const int P = T * (c.k + c.n_shared);     // routed + shared rows in schedule order
   GemmArgs g{};
   g.experts = h->d_experts;
   g.seg_off = h->seg_off;
@@ -376,9 +383,9 @@ qmoe_status qmoe_forward(qmoe_handle* h, const uint16_t* x, int32_t T, uint16_t*
   for (int mat = 0; mat < 2; ++mat) {
     StageTimer tm(h, s, mat == 0 ? QMOE_STAGE_GATE_UP : QMOE_STAGE_DOWN);
     g.mat = mat;
-    g.act = mat == 0 ? x : h->H;
+    g.act = mat == 0 ? h->Xp : h->H;
     g.act_ld = mat == 0 ? c.d : c.I;
-    g.gather = mat == 0 ? h->sorted_token : nullptr;
+    if (mat == 0) QMOE_CUDA(launch_permute_rows(x, h->sorted_token, P, c.d, h->Xp, s), "permute launch");
     g.K = mat == 0 ? c.d : c.I;
     g.MB = mat == 0 ? 2 * c.I / kTileM : c.d / kTileM;
     g.out = mat == 0 ? h->H : h->Y;
@@ -386,7 +393,8 @@ qmoe_status qmoe_forward(qmoe_handle* h, const uint16_t* x, int32_t T, uint16_t*
     for (int fmt = 1; fmt <= 3; ++fmt) {   // one launch per weight format present
       if (!h->fmt_present[fmt]) continue;
       g.tile_off = h->tiles + tile_table_offset(mat, fmt, g.n_seg);
-      QMOE_CUDA(launch_grouped_gemm(g, mat == 0 ? x_map : h->h_map, fmt, bn, h->num_sms, s),
+      QMOE_CUDA(launch_grouped_gemm(g, mat == 0 ? h->xp_map[bn_index(bn)] : h->h_map[bn_index(bn)], fmt, bn,
+                                    h->num_sms, s),
                 mat == 0 ? "gate/up GEMM launch" : "down GEMM launch");
     }
   }
@@ -452,7 +460,7 @@ int32_t qmoe_launches_per_forward(const qmoe_handle* h, int32_t T) {
   if (!h) return 0;
   int fmts = 0;
   for (int f = 1; f <= 3; ++f) fmts += h->fmt_present[f] ? 1 : 0;
-  return 3 + 2 * fmts;  // router (logits + top-k), schedule, gate/up and down GEMM per format, combine
+  return 4 + 2 * fmts;  // router, schedule, row permutation, gate/up and down GEMM per format, combine
 }
 
 qmoe_status qmoe_destroy(qmoe_handle* h) {

@@ -1,4 +1,5 @@
-// Stage 5: gate-weighted unpermute and combine.
+// Stage 5: gate-weighted unpermute and combine (and, for stage 3, the
+// permutation of the activation rows into schedule order).
 //   out[t] = sum_{j<k} g[t,j] * Y[inv_pos[t,j]] + sum_{s<S} Y[T*k + s*T + t]
 // fp32 accumulation in slot order, then the shared experts (weight 1), one
 // round to bf16 (nearest even) at the end.  ("OmniMoE: An Efficient MoE by
@@ -64,7 +65,27 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
   reinterpret_cast<uint4*>(out + (size_t)t * d)[v] = o;
 }
 
+// Activation rows in schedule order for the gate/up GEMM: one thread per
+// 16-byte vector, so each row is read and written with coalesced accesses.
+__global__ void __launch_bounds__(256) permute_rows_kernel(const uint16_t* __restrict__ x,
+                                                           const int32_t* __restrict__ sorted_token, int P, int d,
+                                                           uint16_t* __restrict__ xp) {
+  const int nvec = d >> 3;
+  const long long gv = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gv >= (long long)P * nvec) return;
+  const int p = (int)(gv / nvec), v = (int)(gv - (long long)p * nvec);
+  const int t = __ldg(sorted_token + p);
+  reinterpret_cast<uint4*>(xp + (size_t)p * d)[v] = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d) + v);
+}
+
 }  // namespace
+
+cudaError_t launch_permute_rows(const uint16_t* x, const int32_t* sorted_token, int P, int d, uint16_t* xp,
+                                cudaStream_t s) {
+  const long long n = (long long)P * (d >> 3);
+  permute_rows_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(x, sorted_token, P, d, xp);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_combine(const uint16_t* Y, const float* gate, const int32_t* inv_pos, int T, int k, int S, int d,
                            uint16_t* out, cudaStream_t s) {

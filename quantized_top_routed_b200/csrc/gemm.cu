@@ -12,9 +12,9 @@
 // Layout of the contraction on the tensor cores (tcgen05, kind::f16, M=128):
 //   A (M x K) = 128 weight rows, dequantised to bf16 by CUDA cores and
 //               written straight into tensor memory (tcgen05.st);
-//   B (N x K) = up to BN rows of the expert's segment (tokens), gathered
-//               from x / H by TMA (tile::gather4) into 128-byte-swizzled
-//               shared memory;
+//   B (N x K) = BN consecutive rows of the expert's segment in the permuted
+//               activations (x rows in schedule order, or H), loaded by TMA
+//               tiles (two per K stage) into 128-byte-swizzled shared memory;
 //   D (M x N) = fp32 accumulators in tensor memory, double buffered.
 // Weights are the M side because an expert usually has few tokens: the
 // weight stream is what the kernel moves.  Raw code tiles arrive by TMA bulk
@@ -31,10 +31,11 @@
 // one launch handles the experts of one weight format.  Warp roles, all
 // synchronised through mbarriers:
 //   warp 0       : TMEM allocation; lane 0 streams raw weight tiles (bulk copy)
-//   warp 1       : lanes issue the B gathers (TMA tile::gather4)
+//   warp 1       : lane 0 issues the B tile loads (TMA)
 //   warp 2       : lane 0 issues the MMAs and the commits
-//   warps 3..10  : dequantise A into TMEM; warp w owns TMEM lane quarter
-//                  w % 4 and one 64-wide half of every 128-wide K stage
+//   warps 3..10  : dequantise A into TMEM, as 2 groups of 4 warps that take
+//                  alternate K stages (so two stages are in flight); warp w
+//                  owns TMEM lane quarter w % 4, one weight row per thread
 //   warps 11..14 : epilogue (TMEM -> registers -> scales / SwiGLU -> bf16)
 // Every wait is bounded: a role that waits ~1 s raises an abort flag, all
 // roles drain what they issued, TMEM is freed and the error word is set.
@@ -48,7 +49,9 @@ namespace qmoe {
 namespace {
 
 constexpr int kNDQ = 8;                        // dequantisation warps
-constexpr int kKW = kBK / (kNDQ / 4);          // K elements one dequant thread converts per stage (64)
+constexpr int kGroups = kNDQ / 4;              // groups of 4 warps; group g converts stages g, g+G, ...
+constexpr int kKW = kBK;                       // K elements one dequant thread converts per stage (its row)
+constexpr int kHalf = kKW / 2;                 // converted and stored in two halves
 constexpr int kRawWarp = 0, kBWarp = 1, kMmaWarp = 2;
 constexpr int kDQWarp0 = 3;
 constexpr int kEpiWarp0 = kDQWarp0 + kNDQ;
@@ -59,7 +62,7 @@ constexpr uint32_t kTmemCols = 512;
 template <int FMT>
 struct FmtCfg {
   static constexpr int SB = FMT == QMOE_W_INT4_G128 ? 128 * 64 + 256 : 128 * 128;  // bytes of a raw tile
-  static constexpr int NC = FMT == QMOE_W_INT4_G128 ? kKW / 32 : kKW / 16;          // 16-byte chunks per thread
+  static constexpr int NC = FMT == QMOE_W_INT4_G128 ? kHalf / 32 : kHalf / 16;      // 16-byte chunks per half row
 };
 
 template <int BN, int FMT>
@@ -149,7 +152,7 @@ __device__ __forceinline__ void deq_fp8_word(uint32_t w, uint32_t* o) {
   o[1] = bf2_mul(hi, 0x7B807B80u);
 }
 
-// This thread's 16-byte chunks (K order) -> kKW / 2 bf16 pairs.
+// This thread's 16-byte chunks (K order) -> kHalf / 2 bf16 pairs.
 template <int FMT>
 __device__ __forceinline__ void dequant_slice(const uint4 (&w)[FmtCfg<FMT>::NC], uint32_t sbits, uint32_t* av) {
 #pragma unroll
@@ -181,14 +184,13 @@ __device__ __forceinline__ uint16_t f2bf(float f) {
   return *reinterpret_cast<const uint16_t*>(&b);
 }
 
-// TMA: 4 rows (arbitrary row indices) x 64 bf16 columns of a row-major
-// matrix into 512 bytes of 128-byte-swizzled shared memory.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, int col, int r0, int r1, int r2,
-                                            int r3, uint64_t* bar) {
+// TMA: a box of 64 bf16 columns x BN rows of a row-major matrix into
+// 128-byte-swizzled shared memory (rows past the matrix read as zero).
+__device__ __forceinline__ void tma_tile2d(uint32_t dst, const CUtensorMap* map, int col, int row, uint64_t* bar) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(row), "r"(smem_u32(bar))
       : "memory");
 }
 
@@ -234,12 +236,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (tid == 0) {
     for (int s = 0; s < C::SA; ++s) {
-      mbar_init(&full[s], 1 + kNDQ);   // B producer expect_tx + one arrival per dequant warp
+      mbar_init(&full[s], 1 + 4);      // B producer expect_tx + one arrival per warp of a dequant group
       mbar_init(&empty[s], 1);
     }
     for (int r = 0; r < C::R; ++r) {
       mbar_init(&raw_full[r], 1);
-      mbar_init(&raw_empty[r], kNDQ);
+      mbar_init(&raw_empty[r], 4);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -283,28 +285,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp == kBWarp) {
-    // ---------------- B rows: TMA gathers of the tile's tokens ----------------
+    // ---------------- B rows: two TMA tiles per K stage ----------------
     uint32_t sc = 0, s = 0, ph = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
       const Tile t = decode_tile(tile, tab_off, s_seg_off, s_seg_cnt, n_seg, BN);
-      const int groups = (t.nvalid + 3) >> 2;            // 4-row gathers per K atom
-      int rr[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {                       // lane l gathers rows 4l .. 4l+3
-        const int n = 4 * lane + j;
-        const int p = t.row0 + (n < t.nvalid ? n : 0);
-        rr[j] = (lane < groups) ? (a.gather ? a.gather[p] : p) : 0;
-      }
       for (int ks = 0; ks < KS; ++ks) {
         ok = warp_wait(&empty[s], ph ^ 1, abort_flag);
         if (!ok) break;
-        if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)groups * 4 * 256);
-        __syncwarp();
-        if (lane < groups) {
-          const uint32_t dst = smem_u32(sB + s * C::B_STAGE) + lane * 512;
-          tma_gather4(dst, &act_map, ks * kBK, rr[0], rr[1], rr[2], rr[3], &full[s]);
-          tma_gather4(dst + BN * 128, &act_map, ks * kBK + 64, rr[0], rr[1], rr[2], rr[3], &full[s]);
+        if (lane == 0) {
+          const uint32_t dst = smem_u32(sB + s * C::B_STAGE);
+          mbar_arrive_expect_tx(&full[s], (uint32_t)C::B_STAGE);
+          tma_tile2d(dst, &act_map, ks * kBK, t.row0, &full[s]);
+          tma_tile2d(dst + BN * 128, &act_map, ks * kBK + 64, t.row0, &full[s]);
         }
         __syncwarp();
         ++sc;
@@ -363,25 +356,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < kEpiWarp0) {
     // ---------------- A dequantisation into TMEM ----------------
+    // Group g takes the CTA's K stages g, g + G, g + 2G, ...; its ring slots
+    // advance by G per stage.  Each thread converts its whole weight row of
+    // the stage in two halves (register pressure) and stores it to TMEM.
     const int q = warp & 3;                          // TMEM lane quarter
-    const int h = (warp - kDQWarp0) >> 2;            // which half of the K stage
+    const int g = (warp - kDQWarp0) >> 2;            // group
     const int row = 32 * q + lane;                   // weight row of the tile
-    const uint32_t coff = (uint32_t)(h * F::NC) * 2048u + (uint32_t)row * 16u;   // chunk-major raw tile
-    const uint32_t soff = 128u * 64u + (uint32_t)row * 2u;                       // INT4 group scale
-    const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + C::A_COL0 + h * (kKW / 2);
+    const uint32_t coff = (uint32_t)row * 16u;       // chunk-major raw tile
+    const uint32_t soff = 128u * 64u + (uint32_t)row * 2u;   // INT4 group scale
+    const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + C::A_COL0;
     const uint32_t raw0 = smem_u32(sRaw);
-    uint32_t s = 0, ph = 0, r = 0, rph = 0;
-    int left = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) left += KS;
-    while (left > 0) {
+    constexpr int CPH = F::NC;                       // chunks per half row
+    int stages = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) stages += KS;
+    uint32_t s = g, ph = 0, r = g, rph = 0;
+    for (int i = g; i < stages; i += kGroups) {
       if (!warp_wait(&raw_full[r], rph, abort_flag)) break;
       const uint32_t rp = raw0 + r * C::SLOT;
-      uint4 w[F::NC];
+      uint4 w0[CPH], w1[CPH];
 #pragma unroll
-      for (int k = 0; k < F::NC; ++k)
+      for (int k = 0; k < CPH; ++k) {
         asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(w[k].x), "=r"(w[k].y), "=r"(w[k].z), "=r"(w[k].w)
+                     : "=r"(w0[k].x), "=r"(w0[k].y), "=r"(w0[k].z), "=r"(w0[k].w)
                      : "r"(rp + coff + k * 2048));
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w1[k].x), "=r"(w1[k].y), "=r"(w1[k].z), "=r"(w1[k].w)
+                     : "r"(rp + coff + (CPH + k) * 2048));
+      }
       uint32_t sbits = 0;
       if constexpr (FMT == QMOE_W_INT4_G128) {
         unsigned short sv;
@@ -390,18 +391,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&raw_empty[r]);
-      if (++r == (uint32_t)C::R) { r = 0; rph ^= 1; }
-      uint32_t av[kKW / 2];
-      dequant_slice<FMT>(w, sbits, av);
+      r += kGroups;
+      if (r >= (uint32_t)C::R) { r -= C::R; rph ^= 1; }
+      uint32_t av[kHalf / 2];
+      dequant_slice<FMT>(w0, sbits, av);
       if (!warp_wait(&empty[s], ph ^ 1, abort_flag)) break;
+      const uint32_t ta = tbase + s * 64;
 #pragma unroll
-      for (int c = 0; c < kKW / 32; ++c) tmem_st16(tbase + s * 64 + 16 * c, &av[16 * c]);
+      for (int c = 0; c < kHalf / 32; ++c) tmem_st16(ta + 16 * c, &av[16 * c]);
+      dequant_slice<FMT>(w1, sbits, av);
+#pragma unroll
+      for (int c = 0; c < kHalf / 32; ++c) tmem_st16(ta + kHalf / 2 + 16 * c, &av[16 * c]);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&full[s]);
-      if (++s == (uint32_t)C::SA) { s = 0; ph ^= 1; }
-      --left;
+      s += kGroups;
+      if (s >= (uint32_t)C::SA) { s -= C::SA; ph ^= 1; }
     }
   } else {
     // ---------------- epilogue ----------------

@@ -38,9 +38,8 @@ __host__ __device__ inline int stage_bytes(int fmt) {
 struct GemmArgs {
   const ExpertDev* experts;   // [n_seg]
   int mat;                    // 0: gate/up (gated SwiGLU epilogue), 1: down
-  const uint16_t* act;        // B operand rows (bf16): x [T][d] (gathered) or H [P][I]
+  const uint16_t* act;        // B operand rows (bf16) in schedule order: permuted x [P][d] or H [P][I]
   int act_ld;                 // elements per act row
-  const int32_t* gather;      // row -> act row (sorted_token) or nullptr for identity
   const int32_t* seg_off;     // [n_seg] first permuted row of each segment
   const int32_t* seg_cnt;     // [n_seg] rows in each segment
   const int32_t* tile_off;    // [n_seg + 1] prefix sum of tiles per segment
@@ -267,6 +266,10 @@ size_t schedule_scratch_ints(int max_tokens, int E);
 bool gemm_bn_supported(int bn);
 
 cudaError_t launch_grouped_gemm(const GemmArgs& a, const CUtensorMap& act_map, int fmt, int bn, int num_sms,
+                                cudaStream_t s);
+
+// xp[p] = x[sorted_token[p]] for p < P (activation rows in schedule order).
+cudaError_t launch_permute_rows(const uint16_t* x, const int32_t* sorted_token, int P, int d, uint16_t* xp,
                                 cudaStream_t s);
 
 cudaError_t launch_combine(const uint16_t* Y, const float* gate, const int32_t* inv_pos, int T, int k, int S,

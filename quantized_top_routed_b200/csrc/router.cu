@@ -194,11 +194,23 @@ __global__ void __launch_bounds__(kRouterThreads) router_fused_kernel(
   // every load in flight at once), then one warp per token runs the top-k.
   float* zs = reinterpret_cast<float*>(rsm);                   // [RT][E], reuses the pipeline buffers
   const int rows = min(RT, T - t0);
-  for (int v = tid; v < rows * E; v += kRouterThreads) {
-    const int r = v / E, e = v - r * E;
-    float acc = 0.f;
-    for (int s2 = 0; s2 < split; ++s2) acc += __ldcg(zpart + ((size_t)s2 * T + t0 + r) * E + e);
-    zs[v] = bias ? acc + bias[e] : acc;
+  const int nel = rows * E;                                     // the tile's rows are contiguous in zpart
+  constexpr int kPer = RT * 32 * EPL / kRouterThreads;          // elements per thread (E <= 32 * EPL)
+  float acc[kPer];
+#pragma unroll
+  for (int m = 0; m < kPer; ++m) acc[m] = 0.f;
+  for (int s2 = 0; s2 < split; ++s2) {                          // one round trip per slice
+    const float* zp2 = zpart + ((size_t)s2 * T + t0) * E;
+#pragma unroll
+    for (int m = 0; m < kPer; ++m) {
+      const int v = tid + m * kRouterThreads;
+      if (v < nel) acc[m] += __ldcg(zp2 + v);
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < kPer; ++m) {
+    const int v = tid + m * kRouterThreads;
+    if (v < nel) zs[v] = bias ? acc[m] + bias[v % E] : acc[m];
   }
   __syncthreads();
   const int warp = tid >> 5, lane = tid & 31;

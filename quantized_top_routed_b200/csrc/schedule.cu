@@ -42,6 +42,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint32_t bal[32][kMaxE];
   __shared__ int32_t s_cnt[kMaxE + kMaxShared];
   __shared__ int32_t s_off[kMaxE + 1];
+  __shared__ int32_t s_fmt[kMaxE + kMaxShared];
   int32_t* hist = hist_in_smem ? hist_smem : hist_global;   // [C][E]: chunk counts, then chunk bases
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int C = (T + 31) / 32;
@@ -130,6 +131,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     seg_off[e] = e < E ? s_off[e] : P + (e - E) * T;
     seg_cnt[e] = e < E ? s_cnt[e] : T;
   }
+  for (int e = tid; e < n_seg; e += kThreads) s_fmt[e] = seg_fmt[e];
+  __syncthreads();
   if (warp < 6) {                       // warp w: matrix w / 3, format w % 3 + 1
     const int mat = warp / 3, fmt = warp % 3 + 1;
     const int mb = mat == 0 ? mb3 : mb4;
@@ -138,7 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int e0 = 0; e0 < n_seg; e0 += 32) {
       const int e = e0 + lane;
       int t = 0;
-      if (e < n_seg && seg_fmt[e] == fmt) {
+      if (e < n_seg && s_fmt[e] == fmt) {
         const int cnt = e < E ? s_cnt[e] : T;
         t = ((cnt + bn - 1) / bn) * mb;
       }
