@@ -65,6 +65,13 @@ def max_over_ranks(value: float, device=None) -> float:
     return float(t.item())
 
 
+def job_rate(world: int, tokens_per_rank: int, local_ms: float, device=None):
+    """(step ms, whole-job tokens/s): the slowest rank's step time, and every
+    rank's tokens over that time."""
+    ms = max_over_ranks(local_ms, device)
+    return ms, world * tokens_per_rank / (ms / 1e3)
+
+
 def barrier(device=None):
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized():
@@ -241,9 +248,7 @@ def run_ours(args):
     qmoe.qmoe_profile(dl.handle, False)
     qmoe.qmoe_check_error(dl.handle, stream)
     # warm-up steps were profiled as well; per-launch averages use all calls
-    local_ms = sum(times) / len(times)
-    ms = max_over_ranks(local_ms, dev)
-    value = world * T / (ms / 1e3)
+    ms, value = job_rate(world, T, sum(times) / len(times), dev)
 
     # ---- end to end through the host-buffer entry point ----------------------
     x_host = torch.from_numpy(L.x.view(np.int16).copy()).pin_memory()
@@ -255,7 +260,7 @@ def run_ours(args):
     barrier(dev)
     e2e_times = time_steps(e2e_step, args.steps, args.warmup, flush, stream)
     barrier(dev)
-    e2e_ms = max_over_ranks(sum(e2e_times) / len(e2e_times), dev)
+    e2e_ms, e2e_value = job_rate(world, T, sum(e2e_times) / len(e2e_times), dev)
 
     # ---- roofline of the dominant kernel -----------------------------------
     gu_ms = stage_ms["gate_up"] / max(calls, 1)
@@ -287,7 +292,7 @@ def run_ours(args):
                   "tensor_frac": round(layer_flops(L) / (ms / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
                   "stage_ms": {k_: round(v / max(calls, 1), 5) for k_, v in stage_ms.items()}},
         "roofline": roof,
-        "e2e": {"value": round(world * T / (e2e_ms / 1e3), 1), "unit": UNIT,
+        "e2e": {"value": round(e2e_value, 1), "unit": UNIT,
                 "h2d_bytes_per_step": int(T * L.d * 2), "d2h_bytes_per_step": int(T * L.d * 2)},
         "gpu_launches": qmoe.qmoe_launches_per_forward(dl.handle, T) * args.steps,
         "clocks": clk.summary(),
