@@ -156,6 +156,38 @@ qmoe_status qmoe_destroy(qmoe_handle* h);
 /* Thread-local text of the last failure in this thread ("" if none). */
 const char* qmoe_last_error(void);
 
+/* Stage 1 (router logits, softmax, top-k, renormalised gates) without a
+ * handle and without allocating anything.  The method as published has no
+ * counterpart to this call: it exists for callers that cannot allocate
+ * device memory at the point where they route, for example a serving loop
+ * whose memory is entirely held by another allocator (a caching or arena
+ * allocator that owns all of HBM), or one that must not take the device-wide
+ * synchronisation that cudaMalloc / cudaFree imply in the middle of a step.
+ * It computes exactly what qmoe_route computes for topk_idx / topk_gate
+ * from x, with the same kernel.
+ *
+ * x: bf16 [T][d] (device, 16-byte aligned); router_w: fp32 [E][d] (device,
+ * 16-byte aligned); router_bias: fp32 [E] (device) or NULL.  Outputs
+ * (device): topk_idx int32 [T][k], topk_gate fp32 [T][k].  Requires
+ * d % 128 == 0, 1 <= E <= 256, 1 <= k <= min(E, 16), T >= 1 and
+ * T * E <= QMOE_ROUTE_STATIC_MAX_LOGITS; larger sizes are rejected with
+ * QMOE_ERR_INVALID and nothing is enqueued.
+ *
+ * Scratch: the router's partial logits and its per-token-tile counters live
+ * in one fixed library-global device array of QMOE_ROUTE_STATIC_SCRATCH_BYTES
+ * bytes per device (no cudaMalloc, cudaFree or allocating library call is
+ * made).  The counters are cleared with cudaMemsetAsync on `stream` before
+ * each launch.  The array's address is looked up once per device on the
+ * first call (cudaGetSymbolAddress, which may load the module), so make that
+ * first call before any stream capture begins.  Because the scratch is
+ * shared, calls whose work may overlap on the same GPU (different streams,
+ * or different host threads) race and give wrong results: serialise them. */
+#define QMOE_ROUTE_STATIC_MAX_LOGITS (1 << 20)
+#define QMOE_ROUTE_STATIC_SCRATCH_BYTES (4 * (1 << 20) + 4 * (1 << 15))
+qmoe_status qmoe_route_topk_noalloc(const uint16_t* x, const float* router_w, const float* router_bias,
+                                    int32_t T, int32_t d, int32_t E, int32_t k, int32_t* topk_idx,
+                                    float* topk_gate, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -8,6 +8,7 @@
 
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -472,3 +473,70 @@ qmoe_status qmoe_destroy(qmoe_handle* h) {
 }
 
 }  // extern "C"
+
+// ---- routing without a handle and without allocation ------------------------
+// One fixed device array per device holds the router's partial logits and its
+// per-token-tile counters: counters first (one int per 32-token tile), then
+// the partial-logit slices.  Nothing here allocates device memory.
+namespace {
+
+constexpr size_t kNoallocTickets = size_t(1) << 15;            // ints: covers T up to 2^20
+constexpr size_t kNoallocLogits = QMOE_ROUTE_STATIC_MAX_LOGITS;  // floats
+static_assert(QMOE_ROUTE_STATIC_SCRATCH_BYTES == 4 * (kNoallocLogits + kNoallocTickets), "scratch size");
+static __device__ __align__(256) unsigned char g_route_scratch[QMOE_ROUTE_STATIC_SCRATCH_BYTES];
+
+constexpr int kNoallocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kNoallocMaxDevices] = {};
+int g_noalloc_sms[kNoallocMaxDevices] = {};
+
+// Address of this device's copy of the array (looked up once per device).
+qmoe_status noalloc_scratch(void** addr, int* sms) {
+  int dev = 0;
+  QMOE_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= kNoallocMaxDevices) return fail(QMOE_ERR_UNSUPPORTED, "device ordinal out of range");
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    int d2 = 0, n = 0;
+    qmoe_status st = check_device(&d2, &n);
+    if (st != QMOE_OK) return st;
+    void* p = nullptr;
+    QMOE_CUDA(cudaGetSymbolAddress(&p, g_route_scratch), "cudaGetSymbolAddress for the routing scratch");
+    g_noalloc_sms[dev] = n;
+    g_noalloc_addr[dev] = p;
+  }
+  *addr = g_noalloc_addr[dev];
+  *sms = g_noalloc_sms[dev];
+  return QMOE_OK;
+}
+
+}  // namespace
+
+qmoe_status qmoe_route_topk_noalloc(const uint16_t* x, const float* router_w, const float* router_bias, int32_t T,
+                                    int32_t d, int32_t E, int32_t k, int32_t* topk_idx, float* topk_gate,
+                                    void* stream) {
+  if (!x || !router_w || !topk_idx || !topk_gate)
+    return fail(QMOE_ERR_INVALID, "x, router_w, topk_idx and topk_gate must be non-NULL");
+  if (!aligned16(x) || !aligned16(router_w)) return fail(QMOE_ERR_INVALID, "x and router_w must be 16-byte aligned");
+  if (d < kBK || d % kBK != 0) return fail(QMOE_ERR_INVALID, "d must be a positive multiple of 128");
+  if (E < 1 || E > kMaxE) return fail(QMOE_ERR_INVALID, "E must be in [1, 256]");
+  if (k < 1 || k > E || k > kMaxK) return fail(QMOE_ERR_INVALID, "k must be in [1, min(E, 16)]");
+  if (T < 1) return fail(QMOE_ERR_INVALID, "T must be >= 1");
+  if ((long long)T * E > (long long)kNoallocLogits)
+    return fail(QMOE_ERR_INVALID, "T*E=" + std::to_string((long long)T * E) + " exceeds the fixed routing scratch (" +
+                                      std::to_string(kNoallocLogits) + " logits)");
+  void* base = nullptr;
+  int sms = 0;
+  qmoe_status st = noalloc_scratch(&base, &sms);
+  if (st != QMOE_OK) return st;
+  int* tickets = static_cast<int*>(base);
+  float* zpart = reinterpret_cast<float*>(static_cast<int*>(base) + kNoallocTickets);
+  int split = router_split(T, d, E, sms);
+  while (split > 1 && (long long)split * T * E > (long long)kNoallocLogits) split >>= 1;
+  const int ntick = router_tickets(T);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  QMOE_CUDA(cudaMemsetAsync(tickets, 0, sizeof(int) * (size_t)ntick, s), "clear routing counters");
+  QMOE_CUDA(launch_router(x, router_w, router_bias, T, d, E, k, split, zpart, tickets, topk_idx, topk_gate, s),
+            "router launch");
+  return QMOE_OK;
+}

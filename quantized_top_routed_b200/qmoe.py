@@ -32,7 +32,7 @@ STAGES = ("router", "schedule", "gate_up", "down", "combine")
 
 EXPORTS = ("qmoe_create", "qmoe_route", "qmoe_forward", "qmoe_forward_host", "qmoe_check_error",
            "qmoe_profile", "qmoe_profile_read", "qmoe_launches_per_forward", "qmoe_destroy",
-           "qmoe_last_error")
+           "qmoe_last_error", "qmoe_route_topk_noalloc")
 
 
 class QmoeError(RuntimeError):
@@ -82,8 +82,9 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.qmoe_destroy.argtypes = [vp]
     lib.qmoe_last_error.argtypes = []
     lib.qmoe_last_error.restype = ctypes.c_char_p
+    lib.qmoe_route_topk_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp]
     for name in ("qmoe_create", "qmoe_route", "qmoe_forward", "qmoe_forward_host", "qmoe_check_error",
-                 "qmoe_profile", "qmoe_profile_read", "qmoe_destroy"):
+                 "qmoe_profile", "qmoe_profile_read", "qmoe_destroy", "qmoe_route_topk_noalloc"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -167,6 +168,19 @@ def qmoe_launches_per_forward(h: int, T: int) -> int:
 
 def qmoe_destroy(h: Optional[int]):
     _check(load().qmoe_destroy(h))
+
+
+# Sizes the no-allocation router accepts (T * E logits at most).
+QMOE_ROUTE_STATIC_MAX_LOGITS = 1 << 20
+
+
+def qmoe_route_topk_noalloc(x, router_w, router_bias, T: int, d: int, E: int, k: int, topk_idx, topk_gate,
+                            stream=None):
+    """Router stage without a handle, using the library's fixed scratch
+    array instead of allocating (for callers that cannot allocate device
+    memory mid-step).  Calls that may overlap on one GPU race."""
+    _check(load().qmoe_route_topk_noalloc(_ptr(x), _ptr(router_w), _ptr(router_bias), T, d, E, k,
+                                          _ptr(topk_idx), _ptr(topk_gate), _stream(stream)))
 
 
 # ---------------------------------------------------------------------------

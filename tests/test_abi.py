@@ -86,3 +86,18 @@ def test_calls_reject_null_handle():
         qmoe.qmoe_route(None, 16, None, 4, 16, 16, 16, 16, 16, 16)
     with pytest.raises(qmoe.QmoeError):
         qmoe.qmoe_check_error(None)
+
+
+@pytest.mark.parametrize("T,d,E,k,why", [
+    (0, 256, 8, 2, "T must be"),
+    (4, 200, 8, 2, "multiple of 128"),
+    (4, 256, 300, 2, "E must be"),
+    (4, 256, 8, 9, "k must be"),
+    (qmoe.QMOE_ROUTE_STATIC_MAX_LOGITS // 8 + 1, 256, 8, 2, "exceeds the fixed routing scratch"),
+])
+def test_noalloc_route_validates_before_touching_the_device(T, d, E, k, why):
+    # fake (never dereferenced) pointers: validation rejects before any CUDA call
+    with pytest.raises(qmoe.QmoeError) as ei:
+        qmoe.qmoe_route_topk_noalloc(16, 16, None, T, d, E, k, 16, 16)
+    assert ei.value.status == qmoe.QMOE_ERR_INVALID
+    assert why in str(ei.value)
