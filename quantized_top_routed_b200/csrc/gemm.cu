@@ -28,15 +28,20 @@
 //
 // Persistent CTAs (one per SM) walk the tile list (segment, 128-row weight
 // block, BN-row token block) built on the device by the schedule kernel;
-// one launch handles the experts of one weight format.  Warp roles, all
-// synchronised through mbarriers:
+// one launch handles the experts of one weight format.  A CTA works on G
+// tiles at a time (G = 2 when the accumulators leave TMEM room, BN <= 64):
+// their K stages are interleaved (tile 0 stage k, tile 1 stage k, tile 0
+// stage k+1, ...) and each tile has its own MMA warp and accumulator, so one
+// warp's barrier wait and commit overlap the other warp's MMAs -- a single
+// issuing thread leaves the tensor pipe idle for several hundred cycles per
+// stage.  Warp roles, all synchronised through mbarriers:
 //   warp 0       : TMEM allocation; lane 0 streams raw weight tiles (bulk copy)
 //   warp 1       : lane 0 issues the B tile loads (TMA)
-//   warp 2       : lane 0 issues the MMAs and the commits
-//   warps 3..10  : dequantise A into TMEM, as 2 groups of 4 warps that take
+//   warps 2, 3   : lane 0 of warp 2 + j issues the MMAs and commits of tile j
+//   warps 4..11  : dequantise A into TMEM, as 2 groups of 4 warps that take
 //                  alternate K stages (so two stages are in flight); warp w
 //                  owns TMEM lane quarter w % 4, one weight row per thread
-//   warps 11..14 : epilogue (TMEM -> registers -> scales / SwiGLU -> bf16)
+//   warps 12..15 : epilogue (TMEM -> registers -> scales / SwiGLU -> bf16)
 // Every wait is bounded: a role that waits ~1 s raises an abort flag, all
 // roles drain what they issued, TMEM is freed and the error word is set.
 #include <cuda.h>
@@ -52,8 +57,9 @@ constexpr int kNDQ = 8;                        // dequantisation warps
 constexpr int kGroups = kNDQ / 4;              // groups of 4 warps; group g converts stages g, g+G, ...
 constexpr int kKW = kBK;                       // K elements one dequant thread converts per stage (its row)
 constexpr int kHalf = kKW / 2;                 // converted and stored in two halves
-constexpr int kRawWarp = 0, kBWarp = 1, kMmaWarp = 2;
-constexpr int kDQWarp0 = 3;
+constexpr int kRawWarp = 0, kBWarp = 1, kMmaWarp0 = 2;
+constexpr int kMaxG = 2;                       // tiles in flight per CTA (one MMA warp each)
+constexpr int kDQWarp0 = kMmaWarp0 + kMaxG;
 constexpr int kEpiWarp0 = kDQWarp0 + kNDQ;
 constexpr int kThreads = 32 * (kEpiWarp0 + 4);
 constexpr int kTabMax = kMaxE + kMaxShared + 1;
@@ -67,10 +73,12 @@ struct FmtCfg {
 
 template <int BN, int FMT>
 struct Cfg {
-  static constexpr int SA = BN >= 128 ? 4 : (BN >= 64 ? 6 : 7);   // A/B stages (TMEM + smem)
+  static constexpr int G = BN <= 64 ? 2 : 1;                      // tiles in flight
+  static constexpr int A_COL0 = 2 * G * BN;                       // TMEM: 2 accumulators per tile, then A
+  static constexpr int SA0 = ((int)kTmemCols - A_COL0) / 64;
+  static constexpr int SA = SA0 > 7 ? 7 : SA0;                    // A/B stages (TMEM + smem)
   static constexpr int B_STAGE = BN * 256;                        // BN rows x 128 K bf16
   static constexpr int STAGING = BN * 256;                        // epilogue staging
-  static constexpr int A_COL0 = 2 * BN;                           // TMEM: acc0, acc1, then A stages
   static constexpr int SLOT = (FmtCfg<FMT>::SB + 127) & ~127;     // raw ring slot
   static constexpr int FIXED = SA * B_STAGE + STAGING + 6 * 1024;
   static constexpr int R0 = (224 * 1024 - FIXED) / SLOT;
@@ -80,10 +88,11 @@ struct Cfg {
   static constexpr int OFF_STG = OFF_RAW + R * SLOT;
   static constexpr int OFF_TAB = OFF_STG + STAGING;
   static constexpr int OFF_BAR = (OFF_TAB + 3 * kTabMax * 4 + 127) & ~127;
-  static constexpr int NUM_BARS = 2 * SA + 2 * R + 4 + 1;
+  static constexpr int NUM_BARS = 2 * SA + 2 * R + 4 * G + G;
   static constexpr int OFF_MISC = (OFF_BAR + NUM_BARS * 8 + 15) & ~15;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;               // + alignment slack
-  static_assert(R >= 3, "raw ring too shallow");
+  static_assert(R >= 3 && SA >= 3, "rings too shallow");
+  static_assert(G <= kMaxG, "MMA warps");
   static_assert(A_COL0 + SA * 64 <= (int)kTmemCols, "TMEM budget");
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(B_STAGE % 1024 == 0 && OFF_RAW % 1024 == 0 && OFF_BAR % 8 == 0 && OFF_MISC % 16 == 0,
@@ -204,6 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap act_map) {
   using C = Cfg<BN, FMT>;
   using F = FmtCfg<FMT>;
+  constexpr int G = C::G;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sB = smem + C::OFF_B;
@@ -217,9 +227,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = full + C::SA;             // [SA] MMA done with stage
   uint64_t* raw_full = empty + C::SA;         // [R] raw tile landed
   uint64_t* raw_empty = raw_full + C::R;      // [R] raw tile consumed
-  uint64_t* acc_full = raw_empty + C::R;      // [2]
-  uint64_t* acc_empty = acc_full + 2;         // [2]
-  uint64_t* drain = acc_empty + 2;            // [1]
+  uint64_t* acc_full = raw_empty + C::R;      // [G][2] accumulator of tile lane j, buffer b
+  uint64_t* acc_empty = acc_full + 2 * G;     // [G][2]
+  uint64_t* drain = acc_empty + 2 * G;        // [G]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -243,11 +253,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&raw_full[r], 1);
       mbar_init(&raw_empty[r], 4);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < 2 * G; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 4);     // one arrival per epilogue warp
     }
-    mbar_init(drain, 1);
+    for (int j = 0; j < G; ++j) mbar_init(&drain[j], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -257,25 +267,40 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total = tab_off[n_seg];
+  // This CTA's tiles: blockIdx.x + i * gridDim.x for i < nt, taken G at a time.
+  // Stage order inside a group of gq tiles: for ks, for j < gq: (tile j, ks).
+  const int nt = (int)blockIdx.x < total ? (total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+  auto tile_of = [&](int i) { return decode_tile((int)blockIdx.x + i * (int)gridDim.x, tab_off, s_seg_off,
+                                                 s_seg_cnt, n_seg, BN); };
 
   if (warp == kRawWarp) {
     // ---------------- raw weight tiles: one bulk copy per K stage ----------------
     uint32_t rc = 0, r = 0, ph = 0;         // copies issued, ring slot, slot parity
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-      const Tile t = decode_tile(tile, tab_off, s_seg_off, s_seg_cnt, n_seg, BN);
-      const uint8_t* src = a.experts[t.seg].w[MAT] + (size_t)t.mb * KS * F::SB;
-      for (int ks = 0; ks < KS; ++ks) {
-        ok = warp_wait(&raw_empty[r], ph ^ 1, abort_flag);
-        if (!ok) break;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&raw_full[r], F::SB);
-          bulk_g2s(sRaw + r * C::SLOT, src, F::SB, &raw_full[r]);
+    for (int q0 = 0; q0 < nt && ok; q0 += G) {
+      const int gq = min(G, nt - q0);
+      const uint8_t* src[G];
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        if (j < gq) {
+          const Tile t = tile_of(q0 + j);
+          src[j] = a.experts[t.seg].w[MAT] + (size_t)t.mb * KS * F::SB;
         }
-        __syncwarp();
-        src += F::SB;
-        ++rc;
-        if (++r == (uint32_t)C::R) { r = 0; ph ^= 1; }
+      }
+      for (int ks = 0; ks < KS && ok; ++ks) {
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+          if (j >= gq) break;
+          ok = warp_wait(&raw_empty[r], ph ^ 1, abort_flag);
+          if (!ok) break;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&raw_full[r], F::SB);
+            bulk_g2s(sRaw + r * C::SLOT, src[j] + (size_t)ks * F::SB, F::SB, &raw_full[r]);
+          }
+          __syncwarp();
+          ++rc;
+          if (++r == (uint32_t)C::R) { r = 0; ph ^= 1; }
+        }
       }
     }
     // wait for copies that may still be in flight before the CTA can exit
@@ -288,20 +313,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- B rows: two TMA tiles per K stage ----------------
     uint32_t sc = 0, s = 0, ph = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-      const Tile t = decode_tile(tile, tab_off, s_seg_off, s_seg_cnt, n_seg, BN);
-      for (int ks = 0; ks < KS; ++ks) {
-        ok = warp_wait(&empty[s], ph ^ 1, abort_flag);
-        if (!ok) break;
-        if (lane == 0) {
-          const uint32_t dst = smem_u32(sB + s * C::B_STAGE);
-          mbar_arrive_expect_tx(&full[s], (uint32_t)C::B_STAGE);
-          tma_tile2d(dst, &act_map, ks * kBK, t.row0, &full[s]);
-          tma_tile2d(dst + BN * 128, &act_map, ks * kBK + 64, t.row0, &full[s]);
+    for (int q0 = 0; q0 < nt && ok; q0 += G) {
+      const int gq = min(G, nt - q0);
+      int row0[G];
+#pragma unroll
+      for (int j = 0; j < G; ++j) row0[j] = j < gq ? tile_of(q0 + j).row0 : 0;
+      for (int ks = 0; ks < KS && ok; ++ks) {
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+          if (j >= gq) break;
+          ok = warp_wait(&empty[s], ph ^ 1, abort_flag);
+          if (!ok) break;
+          if (lane == 0) {
+            const uint32_t dst = smem_u32(sB + s * C::B_STAGE);
+            mbar_arrive_expect_tx(&full[s], (uint32_t)C::B_STAGE);
+            tma_tile2d(dst, &act_map, ks * kBK, row0[j], &full[s]);
+            tma_tile2d(dst + BN * 128, &act_map, ks * kBK + 64, row0[j], &full[s]);
+          }
+          __syncwarp();
+          ++sc;
+          if (++s == (uint32_t)C::SA) { s = 0; ph ^= 1; }
         }
-        __syncwarp();
-        ++sc;
-        if (++s == (uint32_t)C::SA) { s = 0; ph ^= 1; }
       }
     }
     if (lane == 0) {
@@ -309,26 +341,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (uint32_t i = first; i < sc; ++i) mbar_wait_drain(&full[i % C::SA], (i / C::SA) & 1);
     }
     __syncwarp();
-  } else if (warp == kMmaWarp) {
-    // ---------------- MMA issuer ----------------
-    uint32_t s = 0, ph = 0, tc = 0;
-    const uint64_t bdesc0 = smem_desc_sw128(smem_u32(sB));
-    const uint32_t a_tmem0 = tmem_base + C::A_COL0;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++tc) {
-      const Tile t = decode_tile(tile, tab_off, s_seg_off, s_seg_cnt, n_seg, BN);
-      const int b = tc & 1;
-      ok = warp_wait(&acc_empty[b], ((tc >> 1) & 1) ^ 1, abort_flag);
-      if (!ok) break;
-      tc_fence_after();
-      const int n_mma = max(16, (t.nvalid + 15) & ~15);
-      const uint32_t idesc = idesc_bf16_m128(n_mma);
-      const uint32_t d_tmem = tmem_base + b * BN;
-      for (int ks = 0; ks < KS; ++ks) {
-        ok = warp_wait(&full[s], ph, abort_flag);
+  } else if (warp < kDQWarp0) {
+    // ---------------- MMA issuer of tile lane j (lane 0 alone) ----------------
+    // A tight single-thread loop: the tensor pipe takes the next MMA only when
+    // the previous one is nearly done, so any work between MMAs is exposed.
+    const int j = warp - kMmaWarp0;
+    if (j < G && lane == 0) {
+      const uint64_t bdesc0 = smem_desc_sw128(smem_u32(sB));
+      const uint32_t a_tmem0 = tmem_base + C::A_COL0;
+      bool ok = true;
+      for (int q0 = 0, q = 0; q0 < nt && ok; q0 += G, ++q) {
+        const int gq = min(G, nt - q0);
+        if (j >= gq) break;
+        const Tile t = tile_of(q0 + j);
+        const int b = q & 1;
+        ok = mbar_wait(&acc_empty[2 * j + b], ((q >> 1) & 1) ^ 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        if (lane == 0) {
+        const uint32_t idesc = idesc_bf16_m128(max(16, (t.nvalid + 15) & ~15));
+        const uint32_t d_tmem = tmem_base + (uint32_t)((2 * j + b) * BN);
+        const int i0 = q0 * KS + j;            // sequence index of this tile's first stage
+        uint32_t s = (uint32_t)(i0 % C::SA), ph = (uint32_t)((i0 / C::SA) & 1);
+        for (int ks = 0; ks < KS; ++ks) {
+          if (!mbar_wait(&full[s], ph, abort_flag)) { ok = false; break; }
+          tc_fence_after();
           // Descriptors of this stage: only the start-address field moves
           // (16-byte units), so each MMA's operands are one add away.
           const uint64_t bdesc = bdesc0 + (uint64_t)(s * (C::B_STAGE >> 4));
@@ -338,27 +374,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_bf16_ts(d_tmem, a_tmem + kk * 8, bdesc + (uint64_t)((kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2),
                         idesc, (ks | kk) != 0);
           mma_commit(&empty[s]);
+          s += gq;
+          if (s >= (uint32_t)C::SA) { s -= C::SA; ph ^= 1; }
         }
-        __syncwarp();
-        if (++s == (uint32_t)C::SA) { s = 0; ph ^= 1; }
+        if (!ok) break;
+        mma_commit(&acc_full[2 * j + b]);
       }
-      if (!ok) break;
-      if (lane == 0) mma_commit(&acc_full[b]);
-      __syncwarp();
-    }
-    if (!ok) {
-      // let every MMA issued so far finish before TMEM is released
-      if (lane == 0) {
-        mma_commit(drain);
-        mbar_wait_drain(drain, 0);
+      if (!ok) {
+        // let every MMA issued so far finish before TMEM is released
+        mma_commit(&drain[j]);
+        mbar_wait_drain(&drain[j], 0);
       }
-      __syncwarp();
     }
+    __syncwarp();
   } else if (warp < kEpiWarp0) {
     // ---------------- A dequantisation into TMEM ----------------
-    // Group g takes the CTA's K stages g, g + G, g + 2G, ...; its ring slots
-    // advance by G per stage.  Each thread converts its whole weight row of
-    // the stage in two halves (register pressure) and stores it to TMEM.
+    // Group g takes the CTA's K stages g, g + G, g + 2G, ... of the stage
+    // sequence; its ring slots advance by the group count per stage.  Each
+    // thread converts its whole weight row of the stage in two halves
+    // (register pressure) and stores it to TMEM.
     const int q = warp & 3;                          // TMEM lane quarter
     const int g = (warp - kDQWarp0) >> 2;            // group
     const int row = 32 * q + lane;                   // weight row of the tile
@@ -367,8 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + C::A_COL0;
     const uint32_t raw0 = smem_u32(sRaw);
     constexpr int CPH = F::NC;                       // chunks per half row
-    int stages = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) stages += KS;
+    const int stages = nt * KS;
     uint32_t s = g, ph = 0, r = g, rph = 0;
     for (int i = g; i < stages; i += kGroups) {
       if (!warp_wait(&raw_full[r], rph, abort_flag)) break;
@@ -419,45 +452,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = 32 * q + lane;             // accumulator row = tile weight row
     constexpr int WCOLS = MAT == 0 ? 16 : 32;
     uint16_t* stg = reinterpret_cast<uint16_t*>(sStg) + (size_t)q * BN * WCOLS;
-    uint32_t tc = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++tc) {
-      const Tile t = decode_tile(tile, tab_off, s_seg_off, s_seg_cnt, n_seg, BN);
-      const int b = tc & 1;
-      const ExpertDev& ex = a.experts[t.seg];
-      const float scale = (FMT != QMOE_W_INT4_G128) ? ex.spc[MAT][t.mb * 128 + r] : 1.0f;
-      ok = warp_wait(&acc_full[b], (tc >> 1) & 1, abort_flag);
-      if (!ok) break;
-      tc_fence_after();
-      const int n_mma = max(16, (t.nvalid + 15) & ~15);
-      const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + b * BN;
-      for (int c0 = 0; c0 < n_mma; c0 += 16) {
-        uint32_t v[16];
-        tmem_ld16(taddr + c0, v);
-        tmem_wait_ld();
-        if (MAT == 0) {
+    for (int q0 = 0, grp = 0; q0 < nt && ok; q0 += G, ++grp) {
+      const int gq = min(G, nt - q0);
+      const int b = grp & 1;
+      for (int j = 0; j < gq && ok; ++j) {
+        const Tile t = tile_of(q0 + j);
+        const ExpertDev& ex = a.experts[t.seg];
+        const float scale = (FMT != QMOE_W_INT4_G128) ? ex.spc[MAT][t.mb * 128 + r] : 1.0f;
+        ok = warp_wait(&acc_full[2 * j + b], (grp >> 1) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const int n_mma = max(16, (t.nvalid + 15) & ~15);
+        const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)((2 * j + b) * BN);
+        for (int c0 = 0; c0 < n_mma; c0 += 16) {
+          uint32_t v[16];
+          tmem_ld16(taddr + c0, v);
+          tmem_wait_ld();
+          if (MAT == 0) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float f = __uint_as_float(v[i]) * scale;
-            const float o = __shfl_xor_sync(0xffffffffu, f, 1);   // up value of the same index
-            if ((lane & 1) == 0) stg[(c0 + i) * WCOLS + (lane >> 1)] = f2bf(silu_f(f) * o);
+            for (int i = 0; i < 16; ++i) {
+              const float f = __uint_as_float(v[i]) * scale;
+              const float o = __shfl_xor_sync(0xffffffffu, f, 1);   // up value of the same index
+              if ((lane & 1) == 0) stg[(c0 + i) * WCOLS + (lane >> 1)] = f2bf(silu_f(f) * o);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) stg[(c0 + i) * WCOLS + lane] = f2bf(__uint_as_float(v[i]) * scale);
           }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) stg[(c0 + i) * WCOLS + lane] = f2bf(__uint_as_float(v[i]) * scale);
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[2 * j + b]);
+        constexpr int VPR = WCOLS / 8;         // 16-byte vectors per token row slice
+        const int col0 = MAT == 0 ? t.mb * 64 + q * 16 : t.mb * 128 + q * 32;
+        for (int v = lane; v < t.nvalid * VPR; v += 32) {
+          const int n = v / VPR, c = v % VPR;
+          *reinterpret_cast<uint4*>(a.out + (size_t)(t.row0 + n) * a.out_ld + col0 + c * 8) =
+              *reinterpret_cast<const uint4*>(stg + n * WCOLS + c * 8);
+        }
+        __syncwarp();
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[b]);
-      constexpr int VPR = WCOLS / 8;         // 16-byte vectors per token row slice
-      const int col0 = MAT == 0 ? t.mb * 64 + q * 16 : t.mb * 128 + q * 32;
-      for (int v = lane; v < t.nvalid * VPR; v += 32) {
-        const int n = v / VPR, c = v % VPR;
-        *reinterpret_cast<uint4*>(a.out + (size_t)(t.row0 + n) * a.out_ld + col0 + c * 8) =
-            *reinterpret_cast<const uint4*>(stg + n * WCOLS + c * 8);
-      }
-      __syncwarp();
     }
   }
 
