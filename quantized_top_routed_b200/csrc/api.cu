@@ -374,7 +374,11 @@ qmoe_status qmoe_forward(qmoe_handle* h, const uint16_t* x, int32_t T, uint16_t*
   st = route_impl(h, x, nullptr, T, h->idx, h->gates, h->counts, h->offsets, h->sorted_token, h->inv_pos, true, bn, s);
   if (st != QMOE_OK) return st;
 
-  const int P = T * (c.k + c.n_shared);     // routed + shared rows in schedule order
+  {
+    // x rows in schedule order (the permutation half of stage 2)
+    StageTimer tm(h, s, QMOE_STAGE_SCHEDULE);
+    QMOE_CUDA(launch_permute_rows(x, h->sorted_token, T * (c.k + c.n_shared), c.d, h->Xp, s), "permute launch");
+  }
   GemmArgs g{};
   g.experts = h->d_experts;
   g.seg_off = h->seg_off;
@@ -386,7 +390,6 @@ qmoe_status qmoe_forward(qmoe_handle* h, const uint16_t* x, int32_t T, uint16_t*
     g.mat = mat;
     g.act = mat == 0 ? h->Xp : h->H;
     g.act_ld = mat == 0 ? c.d : c.I;
-    if (mat == 0) QMOE_CUDA(launch_permute_rows(x, h->sorted_token, P, c.d, h->Xp, s), "permute launch");
     g.K = mat == 0 ? c.d : c.I;
     g.MB = mat == 0 ? 2 * c.I / kTileM : c.d / kTileM;
     g.out = mat == 0 ? h->H : h->Y;

@@ -29,17 +29,18 @@
 // Persistent CTAs (one per SM) walk the tile list (segment, 128-row weight
 // block, BN-row token block) built on the device by the schedule kernel;
 // one launch handles the experts of one weight format.  A CTA works on G
-// tiles at a time (G = 2 when the accumulators leave TMEM room, BN <= 64):
-// their K stages are interleaved (tile 0 stage k, tile 1 stage k, tile 0
-// stage k+1, ...) and each tile has its own MMA warp and accumulator, so one
-// warp's barrier wait and commit overlap the other warp's MMAs -- a single
-// issuing thread leaves the tensor pipe idle for several hundred cycles per
-// stage.  Warp roles, all synchronised through mbarriers:
+// tiles at a time (G = 2 for token blocks of up to 32 rows): K stage k of
+// all G tiles forms one super-stage, produced, signalled and released as a
+// unit, and each tile has its own MMA warp and accumulator, so one warp's
+// barrier wait and commit overlap the other warp's MMAs -- a single issuing
+// thread leaves the tensor pipe idle for several hundred cycles per stage,
+// and every barrier operation costs a dequantisation warp ~200 cycles.
+// Warp roles, all synchronised through mbarriers:
 //   warp 0       : TMEM allocation; lane 0 streams raw weight tiles (bulk copy)
 //   warp 1       : lane 0 issues the B tile loads (TMA)
 //   warps 2, 3   : lane 0 of warp 2 + j issues the MMAs and commits of tile j
 //   warps 4..11  : dequantise A into TMEM, as 2 groups of 4 warps that take
-//                  alternate K stages (so two stages are in flight); warp w
+//                  alternate super-stages (so two are in flight); warp w
 //                  owns TMEM lane quarter w % 4, one weight row per thread
 //   warps 12..15 : epilogue (TMEM -> registers -> scales / SwiGLU -> bf16)
 // Every wait is bounded: a role that waits ~1 s raises an abort flag, all
@@ -54,7 +55,7 @@ namespace qmoe {
 namespace {
 
 constexpr int kNDQ = 8;                        // dequantisation warps
-constexpr int kGroups = kNDQ / 4;              // groups of 4 warps; group g converts stages g, g+G, ...
+constexpr int kGroups = kNDQ / 4;              // groups of 4 warps; group g converts super-stages g, g+2, ...
 constexpr int kKW = kBK;                       // K elements one dequant thread converts per stage (its row)
 constexpr int kHalf = kKW / 2;                 // converted and stored in two halves
 constexpr int kRawWarp = 0, kBWarp = 1, kMmaWarp0 = 2;
@@ -64,6 +65,9 @@ constexpr int kEpiWarp0 = kDQWarp0 + kNDQ;
 constexpr int kThreads = 32 * (kEpiWarp0 + 4);
 constexpr int kTabMax = kMaxE + kMaxShared + 1;
 constexpr uint32_t kTmemCols = 512;
+// Poll back-off (ns) of the roles that wait off the critical path: the
+// producers run ahead of the ring and the epilogue waits a whole tile.
+constexpr uint32_t kSleepRaw = 128, kSleepB = 64, kSleepEpi = 256;
 
 template <int FMT>
 struct FmtCfg {
@@ -73,25 +77,27 @@ struct FmtCfg {
 
 template <int BN, int FMT>
 struct Cfg {
-  static constexpr int G = BN <= 64 ? 2 : 1;                      // tiles in flight
+  static constexpr int G = BN <= 32 ? 2 : 1;                      // tiles in flight
   static constexpr int A_COL0 = 2 * G * BN;                       // TMEM: 2 accumulators per tile, then A
   static constexpr int SA0 = ((int)kTmemCols - A_COL0) / 64;
-  static constexpr int SA = SA0 > 7 ? 7 : SA0;                    // A/B stages (TMEM + smem)
+  static constexpr int SP = (SA0 > 7 ? 7 : SA0) / G;              // super-stage slots (G stages each)
+  static constexpr int SA = SP * G;                               // A/B stage slots (TMEM + smem)
   static constexpr int B_STAGE = BN * 256;                        // BN rows x 128 K bf16
   static constexpr int STAGING = BN * 256;                        // epilogue staging
   static constexpr int SLOT = (FmtCfg<FMT>::SB + 127) & ~127;     // raw ring slot
   static constexpr int FIXED = SA * B_STAGE + STAGING + 6 * 1024;
   static constexpr int R0 = (224 * 1024 - FIXED) / SLOT;
-  static constexpr int R = R0 > 16 ? 16 : R0;                     // raw ring depth
+  static constexpr int RP = (R0 > 16 ? 16 : R0) / G;              // raw ring: super-stage slots
+  static constexpr int R = RP * G;                                // raw ring: tile slots
   static constexpr int OFF_B = 0;
   static constexpr int OFF_RAW = OFF_B + SA * B_STAGE;
   static constexpr int OFF_STG = OFF_RAW + R * SLOT;
   static constexpr int OFF_TAB = OFF_STG + STAGING;
   static constexpr int OFF_BAR = (OFF_TAB + 3 * kTabMax * 4 + 127) & ~127;
-  static constexpr int NUM_BARS = 2 * SA + 2 * R + 4 * G + G;
+  static constexpr int NUM_BARS = 2 * SP + 2 * RP + 4 * G + G;
   static constexpr int OFF_MISC = (OFF_BAR + NUM_BARS * 8 + 15) & ~15;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;               // + alignment slack
-  static_assert(R >= 3 && SA >= 3, "rings too shallow");
+  static_assert(RP >= 3 && SP >= 3, "rings too shallow");
   static_assert(G <= kMaxG, "MMA warps");
   static_assert(A_COL0 + SA * 64 <= (int)kTmemCols, "TMEM budget");
   static_assert(SMEM <= 232448, "shared memory budget");
@@ -207,6 +213,10 @@ __device__ __forceinline__ void tma_tile2d(uint32_t dst, const CUtensorMap* map,
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
 }
+// The same for roles off the critical path: back off between polls.
+__device__ __forceinline__ bool warp_wait_backoff(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t ns) {
+  return __all_sync(0xffffffffu, mbar_wait_backoff(bar, parity, abort, ns));
+}
 
 template <int BN, int MAT, int FMT>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -223,11 +233,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   int32_t* s_seg_off = tab_off + kTabMax;
   int32_t* s_seg_cnt = s_seg_off + kTabMax;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* full = bars;                      // [SA] B landed + A in TMEM
-  uint64_t* empty = full + C::SA;             // [SA] MMA done with stage
-  uint64_t* raw_full = empty + C::SA;         // [R] raw tile landed
-  uint64_t* raw_empty = raw_full + C::R;      // [R] raw tile consumed
-  uint64_t* acc_full = raw_empty + C::R;      // [G][2] accumulator of tile lane j, buffer b
+  uint64_t* full = bars;                      // [SP] B landed + A in TMEM, per super-stage
+  uint64_t* empty = full + C::SP;             // [SP] MMAs done with the super-stage
+  uint64_t* raw_full = empty + C::SP;         // [RP] raw tiles of a super-stage landed
+  uint64_t* raw_empty = raw_full + C::RP;     // [RP] raw tiles consumed
+  uint64_t* acc_full = raw_empty + C::RP;     // [G][2] accumulator of tile lane j, buffer b
   uint64_t* acc_empty = acc_full + 2 * G;     // [G][2]
   uint64_t* drain = acc_empty + 2 * G;        // [G]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
@@ -245,11 +255,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   if (tid == 0) {
-    for (int s = 0; s < C::SA; ++s) {
+    for (int s = 0; s < C::SP; ++s) {
       mbar_init(&full[s], 1 + 4);      // B producer expect_tx + one arrival per warp of a dequant group
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], G);         // one commit per tile lane
     }
-    for (int r = 0; r < C::R; ++r) {
+    for (int r = 0; r < C::RP; ++r) {
       mbar_init(&raw_full[r], 1);
       mbar_init(&raw_empty[r], 4);
     }
@@ -267,15 +277,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total = tab_off[n_seg];
-  // This CTA's tiles: blockIdx.x + i * gridDim.x for i < nt, taken G at a time.
-  // Stage order inside a group of gq tiles: for ks, for j < gq: (tile j, ks).
+  // This CTA's tiles: blockIdx.x + i * gridDim.x for i < nt, taken G at a
+  // time.  A group of gq tiles is processed as KS super-stages; super-stage
+  // ks holds K stage ks of every tile of the group (tile j in stage slot j of
+  // the super-stage slot) and is produced, signalled and released as a unit.
   const int nt = (int)blockIdx.x < total ? (total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
   auto tile_of = [&](int i) { return decode_tile((int)blockIdx.x + i * (int)gridDim.x, tab_off, s_seg_off,
                                                  s_seg_cnt, n_seg, BN); };
 
   if (warp == kRawWarp) {
-    // ---------------- raw weight tiles: one bulk copy per K stage ----------------
-    uint32_t rc = 0, r = 0, ph = 0;         // copies issued, ring slot, slot parity
+    // ---------------- raw weight tiles: one bulk copy per tile per K stage ----------------
+    uint32_t rc = 0, r = 0, ph = 0;         // super-stages issued, ring slot, slot parity
     bool ok = true;
     for (int q0 = 0; q0 < nt && ok; q0 += G) {
       const int gq = min(G, nt - q0);
@@ -287,30 +299,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           src[j] = a.experts[t.seg].w[MAT] + (size_t)t.mb * KS * F::SB;
         }
       }
-      for (int ks = 0; ks < KS && ok; ++ks) {
+      for (int ks = 0; ks < KS; ++ks) {
+        ok = warp_wait_backoff(&raw_empty[r], ph ^ 1, abort_flag, kSleepRaw);
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&raw_full[r], (uint32_t)(gq * F::SB));
 #pragma unroll
-        for (int j = 0; j < G; ++j) {
-          if (j >= gq) break;
-          ok = warp_wait(&raw_empty[r], ph ^ 1, abort_flag);
-          if (!ok) break;
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&raw_full[r], F::SB);
-            bulk_g2s(sRaw + r * C::SLOT, src[j] + (size_t)ks * F::SB, F::SB, &raw_full[r]);
-          }
-          __syncwarp();
-          ++rc;
-          if (++r == (uint32_t)C::R) { r = 0; ph ^= 1; }
+          for (int j = 0; j < G; ++j)
+            if (j < gq) bulk_g2s(sRaw + (r * G + j) * C::SLOT, src[j] + (size_t)ks * F::SB, F::SB, &raw_full[r]);
         }
+        __syncwarp();
+        ++rc;
+        if (++r == (uint32_t)C::RP) { r = 0; ph ^= 1; }
       }
     }
     // wait for copies that may still be in flight before the CTA can exit
     if (lane == 0) {
-      const uint32_t first = rc > (uint32_t)C::R ? rc - C::R : 0;
-      for (uint32_t i = first; i < rc; ++i) mbar_wait_drain(&raw_full[i % C::R], (i / C::R) & 1);
+      const uint32_t first = rc > (uint32_t)C::RP ? rc - C::RP : 0;
+      for (uint32_t i = first; i < rc; ++i) mbar_wait_drain(&raw_full[i % C::RP], (i / C::RP) & 1);
     }
     __syncwarp();
   } else if (warp == kBWarp) {
-    // ---------------- B rows: two TMA tiles per K stage ----------------
+    // ---------------- B rows: two TMA tiles per tile per K stage ----------------
     uint32_t sc = 0, s = 0, ph = 0;
     bool ok = true;
     for (int q0 = 0; q0 < nt && ok; q0 += G) {
@@ -318,27 +328,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       int row0[G];
 #pragma unroll
       for (int j = 0; j < G; ++j) row0[j] = j < gq ? tile_of(q0 + j).row0 : 0;
-      for (int ks = 0; ks < KS && ok; ++ks) {
+      for (int ks = 0; ks < KS; ++ks) {
+        ok = warp_wait_backoff(&empty[s], ph ^ 1, abort_flag, kSleepB);
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[s], (uint32_t)(gq * C::B_STAGE));
 #pragma unroll
-        for (int j = 0; j < G; ++j) {
-          if (j >= gq) break;
-          ok = warp_wait(&empty[s], ph ^ 1, abort_flag);
-          if (!ok) break;
-          if (lane == 0) {
-            const uint32_t dst = smem_u32(sB + s * C::B_STAGE);
-            mbar_arrive_expect_tx(&full[s], (uint32_t)C::B_STAGE);
-            tma_tile2d(dst, &act_map, ks * kBK, row0[j], &full[s]);
-            tma_tile2d(dst + BN * 128, &act_map, ks * kBK + 64, row0[j], &full[s]);
+          for (int j = 0; j < G; ++j) {
+            if (j < gq) {
+              const uint32_t dst = smem_u32(sB + (s * G + j) * C::B_STAGE);
+              tma_tile2d(dst, &act_map, ks * kBK, row0[j], &full[s]);
+              tma_tile2d(dst + BN * 128, &act_map, ks * kBK + 64, row0[j], &full[s]);
+            }
           }
-          __syncwarp();
-          ++sc;
-          if (++s == (uint32_t)C::SA) { s = 0; ph ^= 1; }
         }
+        __syncwarp();
+        ++sc;
+        if (++s == (uint32_t)C::SP) { s = 0; ph ^= 1; }
       }
     }
     if (lane == 0) {
-      const uint32_t first = sc > (uint32_t)C::SA ? sc - C::SA : 0;
-      for (uint32_t i = first; i < sc; ++i) mbar_wait_drain(&full[i % C::SA], (i / C::SA) & 1);
+      const uint32_t first = sc > (uint32_t)C::SP ? sc - C::SP : 0;
+      for (uint32_t i = first; i < sc; ++i) mbar_wait_drain(&full[i % C::SP], (i / C::SP) & 1);
     }
     __syncwarp();
   } else if (warp < kDQWarp0) {
@@ -347,8 +358,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the previous one is nearly done, so any work between MMAs is exposed.
     const int j = warp - kMmaWarp0;
     if (j < G && lane == 0) {
-      const uint64_t bdesc0 = smem_desc_sw128(smem_u32(sB));
-      const uint32_t a_tmem0 = tmem_base + C::A_COL0;
+      const uint64_t bdesc0 = smem_desc_sw128(smem_u32(sB + j * C::B_STAGE));
+      const uint32_t a_tmem0 = tmem_base + C::A_COL0 + (uint32_t)(j * 64);
       bool ok = true;
       for (int q0 = 0, q = 0; q0 < nt && ok; q0 += G, ++q) {
         const int gq = min(G, nt - q0);
@@ -360,22 +371,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t idesc = idesc_bf16_m128(max(16, (t.nvalid + 15) & ~15));
         const uint32_t d_tmem = tmem_base + (uint32_t)((2 * j + b) * BN);
-        const int i0 = q0 * KS + j;            // sequence index of this tile's first stage
-        uint32_t s = (uint32_t)(i0 % C::SA), ph = (uint32_t)((i0 / C::SA) & 1);
+        const int u0 = q * KS;                 // super-stage index of this group's first K stage
+        uint32_t s = (uint32_t)(u0 % C::SP), ph = (uint32_t)((u0 / C::SP) & 1);
         for (int ks = 0; ks < KS; ++ks) {
           if (!mbar_wait(&full[s], ph, abort_flag)) { ok = false; break; }
           tc_fence_after();
           // Descriptors of this stage: only the start-address field moves
           // (16-byte units), so each MMA's operands are one add away.
-          const uint64_t bdesc = bdesc0 + (uint64_t)(s * (C::B_STAGE >> 4));
-          const uint32_t a_tmem = a_tmem0 + s * 64;
+          const uint64_t bdesc = bdesc0 + (uint64_t)(s * (G * C::B_STAGE >> 4));
+          const uint32_t a_tmem = a_tmem0 + s * (G * 64);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_bf16_ts(d_tmem, a_tmem + kk * 8, bdesc + (uint64_t)((kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2),
                         idesc, (ks | kk) != 0);
           mma_commit(&empty[s]);
-          s += gq;
-          if (s >= (uint32_t)C::SA) { s -= C::SA; ph ^= 1; }
+          for (int e = gq; e < G; ++e) mma_commit(&empty[s]);   // stand in for absent tile lanes
+          if (++s == (uint32_t)C::SP) { s = 0; ph ^= 1; }
         }
         if (!ok) break;
         mma_commit(&acc_full[2 * j + b]);
@@ -389,10 +400,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp < kEpiWarp0) {
     // ---------------- A dequantisation into TMEM ----------------
-    // Group g takes the CTA's K stages g, g + G, g + 2G, ... of the stage
-    // sequence; its ring slots advance by the group count per stage.  Each
-    // thread converts its whole weight row of the stage in two halves
-    // (register pressure) and stores it to TMEM.
+    // Group g takes super-stages g, g + 2, g + 4, ...: it waits once for the
+    // super-stage's raw tiles and its A slots, converts the gq tiles' K
+    // stage (one weight row per thread, in two halves for register
+    // pressure) into TMEM, and signals once.  A super-stage is published
+    // (full barrier) only after the group's next one has been converted up
+    // to its first store, so the store latency overlaps useful work.  This
+    // cannot deadlock: that step waits only for the MMAs to release the slot
+    // of super-stage u + 2 - SP, an earlier one (SP >= 3).
     const int q = warp & 3;                          // TMEM lane quarter
     const int g = (warp - kDQWarp0) >> 2;            // group
     const int row = 32 * q + lane;                   // weight row of the tile
@@ -401,46 +416,67 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + C::A_COL0;
     const uint32_t raw0 = smem_u32(sRaw);
     constexpr int CPH = F::NC;                       // chunks per half row
-    const int stages = nt * KS;
-    uint32_t s = g, ph = 0, r = g, rph = 0;
-    for (int i = g; i < stages; i += kGroups) {
-      if (!warp_wait(&raw_full[r], rph, abort_flag)) break;
-      const uint32_t rp = raw0 + r * C::SLOT;
-      uint4 w0[CPH], w1[CPH];
+    uint32_t s = 0, ph = 0, r = 0, rph = 0;          // ring positions of super-stage u
+    int pending = -1;                                // A slot whose stores are not yet published
+    bool ok = true;
+    for (int q0 = 0, u = 0; q0 < nt && ok; q0 += G) {
+      const int gq = min(G, nt - q0);
+      for (int ks = 0; ks < KS; ++ks, ++u) {
+        if (u % kGroups == g) {
+          if (!(ok = warp_wait(&raw_full[r], rph, abort_flag))) break;
+          for (int jj = 0; jj < gq; ++jj) {
+            const uint32_t rp = raw0 + (r * G + jj) * C::SLOT;
+            uint4 w0[CPH], w1[CPH];
 #pragma unroll
-      for (int k = 0; k < CPH; ++k) {
-        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(w0[k].x), "=r"(w0[k].y), "=r"(w0[k].z), "=r"(w0[k].w)
-                     : "r"(rp + coff + k * 2048));
-        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(w1[k].x), "=r"(w1[k].y), "=r"(w1[k].z), "=r"(w1[k].w)
-                     : "r"(rp + coff + (CPH + k) * 2048));
+            for (int k = 0; k < CPH; ++k) {
+              asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(w0[k].x), "=r"(w0[k].y), "=r"(w0[k].z), "=r"(w0[k].w)
+                           : "r"(rp + coff + k * 2048));
+              asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(w1[k].x), "=r"(w1[k].y), "=r"(w1[k].z), "=r"(w1[k].w)
+                           : "r"(rp + coff + (CPH + k) * 2048));
+            }
+            uint32_t sbits = 0;
+            if constexpr (FMT == QMOE_W_INT4_G128) {
+              unsigned short sv;
+              asm volatile("ld.shared.u16 %0, [%1];" : "=h"(sv) : "r"(rp + soff));
+              sbits = sv;
+            }
+            uint32_t av[kHalf / 2];
+            dequant_slice<FMT>(w0, sbits, av);
+            if (jj == 0) {
+              if (!(ok = warp_wait(&empty[s], ph ^ 1, abort_flag))) break;
+              tc_fence_after();               // TMEM stores after the MMAs' reads of this slot
+              // The previous super-stage's stores were left in flight while
+              // this one was loaded and converted; complete and publish them.
+              if (pending >= 0) {
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full[pending]);
+              }
+            }
+            const uint32_t ta = tbase + (s * G + jj) * 64;
+#pragma unroll
+            for (int c = 0; c < kHalf / 32; ++c) tmem_st16(ta + 16 * c, &av[16 * c]);
+            dequant_slice<FMT>(w1, sbits, av);
+#pragma unroll
+            for (int c = 0; c < kHalf / 32; ++c) tmem_st16(ta + kHalf / 2 + 16 * c, &av[16 * c]);
+          }
+          if (!ok) break;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&raw_empty[r]);
+          pending = (int)s;
+        }
+        if (++r == (uint32_t)C::RP) { r = 0; rph ^= 1; }
+        if (++s == (uint32_t)C::SP) { s = 0; ph ^= 1; }
       }
-      uint32_t sbits = 0;
-      if constexpr (FMT == QMOE_W_INT4_G128) {
-        unsigned short sv;
-        asm volatile("ld.shared.u16 %0, [%1];" : "=h"(sv) : "r"(rp + soff));
-        sbits = sv;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&raw_empty[r]);
-      r += kGroups;
-      if (r >= (uint32_t)C::R) { r -= C::R; rph ^= 1; }
-      uint32_t av[kHalf / 2];
-      dequant_slice<FMT>(w0, sbits, av);
-      if (!warp_wait(&empty[s], ph ^ 1, abort_flag)) break;
-      const uint32_t ta = tbase + s * 64;
-#pragma unroll
-      for (int c = 0; c < kHalf / 32; ++c) tmem_st16(ta + 16 * c, &av[16 * c]);
-      dequant_slice<FMT>(w1, sbits, av);
-#pragma unroll
-      for (int c = 0; c < kHalf / 32; ++c) tmem_st16(ta + kHalf / 2 + 16 * c, &av[16 * c]);
+    }
+    if (pending >= 0) {
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&full[s]);
-      s += kGroups;
-      if (s >= (uint32_t)C::SA) { s -= C::SA; ph ^= 1; }
+      if (lane == 0) mbar_arrive(&full[pending]);
     }
   } else {
     // ---------------- epilogue ----------------
@@ -460,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Tile t = tile_of(q0 + j);
         const ExpertDev& ex = a.experts[t.seg];
         const float scale = (FMT != QMOE_W_INT4_G128) ? ex.spc[MAT][t.mb * 128 + r] : 1.0f;
-        ok = warp_wait(&acc_full[2 * j + b], (grp >> 1) & 1, abort_flag);
+        ok = warp_wait_backoff(&acc_full[2 * j + b], (grp >> 1) & 1, abort_flag, kSleepEpi);
         if (!ok) break;
         tc_fence_after();
         const int n_mma = max(16, (t.nvalid + 15) & ~15);

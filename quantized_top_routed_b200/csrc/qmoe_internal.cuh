@@ -124,6 +124,28 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   return mbar_wait_slow(addr, parity, abort);
 }
 
+// Bounded wait that sleeps ns nanoseconds between polls: for roles whose
+// waits are long and off the critical path, so that their polling leaves the
+// issue slots to the warps doing the work.
+static __device__ __noinline__ bool mbar_wait_backoff_slow(uint32_t addr, uint32_t parity, volatile int* abort,
+                                                           uint32_t ns) {
+  const long long t0 = clock64();
+  for (;;) {
+    if (mbar_try_wait(addr, parity)) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > (1ll << 31)) {
+      *abort = 1;
+      return false;
+    }
+    __nanosleep(ns);
+  }
+}
+__device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t ns) {
+  const uint32_t addr = smem_u32(bar);
+  if (mbar_try_wait(addr, parity)) return true;
+  return mbar_wait_backoff_slow(addr, parity, abort, ns);
+}
+
 // Same, ignoring the abort flag (used while draining on the way out).
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
   const uint32_t addr = smem_u32(bar);
