@@ -18,6 +18,11 @@ using namespace qmoe;
 
 namespace {
 
+// Programmatic dependent launch of the kernels after the router.  Off: with
+// it on, the mixed-format workload hit an unspecified launch failure whose
+// cause was not found; every kernel still calls pdl_wait(), a no-op here.
+constexpr bool kUsePdl = false;
+
 thread_local std::string g_last_error;
 
 qmoe_status fail(qmoe_status st, const std::string& msg) {
@@ -199,7 +204,7 @@ qmoe_status route_impl(qmoe_handle* h, const uint16_t* x, const float* logits, i
   }
   {
     StageTimer tm(h, s, QMOE_STAGE_SCHEDULE);
-    QMOE_CUDA(launch_schedule(idx, T, c.k, c.E, tables ? c.n_shared : 0, bn, 2 * c.I / kTileM, c.d / kTileM,
+    QMOE_CUDA(launch_schedule(kUsePdl, idx, T, c.k, c.E, tables ? c.n_shared : 0, bn, 2 * c.I / kTileM, c.d / kTileM,
                               h->seg_fmt, counts, offsets, sorted_token, inv_pos, tables ? h->seg_off : nullptr,
                               tables ? h->seg_cnt : nullptr, h->tiles, h->sched_scratch, s),
               "schedule launch");
@@ -377,7 +382,7 @@ qmoe_status qmoe_forward(qmoe_handle* h, const uint16_t* x, int32_t T, uint16_t*
   {
     // x rows in schedule order (the permutation half of stage 2)
     StageTimer tm(h, s, QMOE_STAGE_SCHEDULE);
-    QMOE_CUDA(launch_permute_rows(x, h->sorted_token, T * (c.k + c.n_shared), c.d, h->Xp, s), "permute launch");
+    QMOE_CUDA(launch_permute_rows(kUsePdl, x, h->sorted_token, T * (c.k + c.n_shared), c.d, h->Xp, s), "permute launch");
   }
   GemmArgs g{};
   g.experts = h->d_experts;
@@ -397,14 +402,14 @@ qmoe_status qmoe_forward(qmoe_handle* h, const uint16_t* x, int32_t T, uint16_t*
     for (int fmt = 1; fmt <= 3; ++fmt) {   // one launch per weight format present
       if (!h->fmt_present[fmt]) continue;
       g.tile_off = h->tiles + tile_table_offset(mat, fmt, g.n_seg);
-      QMOE_CUDA(launch_grouped_gemm(g, mat == 0 ? h->xp_map[bn_index(bn)] : h->h_map[bn_index(bn)], fmt, bn,
+      QMOE_CUDA(launch_grouped_gemm(kUsePdl, g, mat == 0 ? h->xp_map[bn_index(bn)] : h->h_map[bn_index(bn)], fmt, bn,
                                     h->num_sms, s),
                 mat == 0 ? "gate/up GEMM launch" : "down GEMM launch");
     }
   }
   {
     StageTimer tm(h, s, QMOE_STAGE_COMBINE);
-    QMOE_CUDA(launch_combine(h->Y, h->gates, h->inv_pos, T, c.k, c.n_shared, c.d, out, s), "combine launch");
+    QMOE_CUDA(launch_combine(kUsePdl, h->Y, h->gates, h->inv_pos, T, c.k, c.n_shared, c.d, out, s), "combine launch");
   }
   if (h->profiling) h->profiled_calls++;
   return QMOE_OK;

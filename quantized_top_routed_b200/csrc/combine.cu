@@ -33,6 +33,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ Y, const float* __restrict__ gate,
                                                       const int32_t* __restrict__ inv_pos, int T, int k, int S,
                                                       int d, uint16_t* __restrict__ out) {
+  pdl_wait();                                   // Y is complete past this point
   const int nvec = d >> 3;
   const long long gv = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (gv >= (long long)T * nvec) return;
@@ -70,6 +71,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
 __global__ void __launch_bounds__(256) permute_rows_kernel(const uint16_t* __restrict__ x,
                                                            const int32_t* __restrict__ sorted_token, int P, int d,
                                                            uint16_t* __restrict__ xp) {
+  pdl_wait();                                   // the schedule's permutation is complete past this point
   const int nvec = d >> 3;
   const long long gv = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (gv >= (long long)P * nvec) return;
@@ -80,18 +82,18 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const uint16_t* __res
 
 }  // namespace
 
-cudaError_t launch_permute_rows(const uint16_t* x, const int32_t* sorted_token, int P, int d, uint16_t* xp,
+cudaError_t launch_permute_rows(bool pdl, const uint16_t* x, const int32_t* sorted_token, int P, int d, uint16_t* xp,
                                 cudaStream_t s) {
   const long long n = (long long)P * (d >> 3);
-  permute_rows_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(x, sorted_token, P, d, xp);
-  return cudaGetLastError();
+  return launch_ex(permute_rows_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, pdl, x, sorted_token, P,
+                   d, xp);
 }
 
-cudaError_t launch_combine(const uint16_t* Y, const float* gate, const int32_t* inv_pos, int T, int k, int S, int d,
+cudaError_t launch_combine(bool pdl, const uint16_t* Y, const float* gate, const int32_t* inv_pos, int T, int k, int S, int d,
                            uint16_t* out, cudaStream_t s) {
   const long long n = (long long)T * (d >> 3);
-  combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(Y, gate, inv_pos, T, k, S, d, out);
-  return cudaGetLastError();
+  return launch_ex(combine_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, pdl, Y, gate, inv_pos, T, k, S,
+                   d, out);
 }
 
 }  // namespace qmoe

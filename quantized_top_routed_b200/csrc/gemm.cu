@@ -247,13 +247,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_seg = a.n_seg;
   const int KS = a.K / kBK;
 
-  for (int i = tid; i <= n_seg; i += kThreads) {
-    tab_off[i] = a.tile_off[i];
-    if (i < n_seg) {
-      s_seg_off[i] = a.seg_off[i];
-      s_seg_cnt[i] = a.seg_cnt[i];
-    }
-  }
   if (tid == 0) {
     for (int s = 0; s < C::SP; ++s) {
       mbar_init(&full[s], 1 + 4);      // B producer expect_tx + one arrival per warp of a dequant group
@@ -272,6 +265,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
   }
   if (warp == kRawWarp) tmem_alloc(tmem_slot, kTmemCols);
+  // Everything above is private to the CTA and may overlap the previous
+  // kernel's tail; the tile tables and the activations are read only after
+  // that kernel has completed.
+  pdl_wait();
+  for (int i = tid; i <= n_seg; i += kThreads) {
+    tab_off[i] = a.tile_off[i];
+    if (i < n_seg) {
+      s_seg_off[i] = a.seg_off[i];
+      s_seg_cnt[i] = a.seg_cnt[i];
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -542,41 +546,40 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int BN, int MAT, int FMT>
-cudaError_t launch_one(const GemmArgs& a, const CUtensorMap& map, int num_sms, cudaStream_t s) {
+cudaError_t launch_one(bool pdl, const GemmArgs& a, const CUtensorMap& map, int num_sms, cudaStream_t s) {
   using C = Cfg<BN, FMT>;
   auto kern = grouped_gemm_kernel<BN, MAT, FMT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<num_sms, kThreads, C::SMEM, s>>>(a, map);
-  return cudaGetLastError();
+  return launch_ex(kern, dim3(num_sms), dim3(kThreads), C::SMEM, s, pdl, a, map);
 }
 
 template <int BN, int MAT>
-cudaError_t launch_fmt(const GemmArgs& a, const CUtensorMap& map, int fmt, int num_sms, cudaStream_t s) {
+cudaError_t launch_fmt(bool pdl, const GemmArgs& a, const CUtensorMap& map, int fmt, int num_sms, cudaStream_t s) {
   switch (fmt) {
-    case QMOE_W_INT4_G128: return launch_one<BN, MAT, QMOE_W_INT4_G128>(a, map, num_sms, s);
-    case QMOE_W_FP8_E4M3_PC: return launch_one<BN, MAT, QMOE_W_FP8_E4M3_PC>(a, map, num_sms, s);
-    case QMOE_W_INT8_PC: return launch_one<BN, MAT, QMOE_W_INT8_PC>(a, map, num_sms, s);
+    case QMOE_W_INT4_G128: return launch_one<BN, MAT, QMOE_W_INT4_G128>(pdl, a, map, num_sms, s);
+    case QMOE_W_FP8_E4M3_PC: return launch_one<BN, MAT, QMOE_W_FP8_E4M3_PC>(pdl, a, map, num_sms, s);
+    case QMOE_W_INT8_PC: return launch_one<BN, MAT, QMOE_W_INT8_PC>(pdl, a, map, num_sms, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
 template <int BN>
-cudaError_t launch_bn(const GemmArgs& a, const CUtensorMap& map, int fmt, int num_sms, cudaStream_t s) {
-  return a.mat == 0 ? launch_fmt<BN, 0>(a, map, fmt, num_sms, s) : launch_fmt<BN, 1>(a, map, fmt, num_sms, s);
+cudaError_t launch_bn(bool pdl, const GemmArgs& a, const CUtensorMap& map, int fmt, int num_sms, cudaStream_t s) {
+  return a.mat == 0 ? launch_fmt<BN, 0>(pdl, a, map, fmt, num_sms, s) : launch_fmt<BN, 1>(pdl, a, map, fmt, num_sms, s);
 }
 
 }  // namespace
 
 bool gemm_bn_supported(int bn) { return bn == 16 || bn == 32 || bn == 64 || bn == 128; }
 
-cudaError_t launch_grouped_gemm(const GemmArgs& a, const CUtensorMap& act_map, int fmt, int bn, int num_sms,
+cudaError_t launch_grouped_gemm(bool pdl, const GemmArgs& a, const CUtensorMap& act_map, int fmt, int bn, int num_sms,
                                 cudaStream_t s) {
   switch (bn) {
-    case 16: return launch_bn<16>(a, act_map, fmt, num_sms, s);
-    case 32: return launch_bn<32>(a, act_map, fmt, num_sms, s);
-    case 64: return launch_bn<64>(a, act_map, fmt, num_sms, s);
-    case 128: return launch_bn<128>(a, act_map, fmt, num_sms, s);
+    case 16: return launch_bn<16>(pdl, a, act_map, fmt, num_sms, s);
+    case 32: return launch_bn<32>(pdl, a, act_map, fmt, num_sms, s);
+    case 64: return launch_bn<64>(pdl, a, act_map, fmt, num_sms, s);
+    case 128: return launch_bn<128>(pdl, a, act_map, fmt, num_sms, s);
     default: return cudaErrorInvalidValue;
   }
 }

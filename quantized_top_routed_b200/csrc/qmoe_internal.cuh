@@ -184,6 +184,13 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// --- programmatic dependent launch ------------------------------------------
+// A kernel launched with launch_ex(pdl = true) may start while its
+// predecessor on the stream is finishing; pdl_wait() blocks until that
+// predecessor has completed and its memory is visible, so every kernel calls
+// it before reading what the previous kernel wrote.  (A no-op without PDL.)
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // --- tcgen05 ---------------------------------------------------------------
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -266,6 +273,24 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
 // ---------------------------------------------------------------------------
 // host-side launchers (implemented in the .cu files)
 // ---------------------------------------------------------------------------
+// Launch kern<<<grid, block, smem, s>>>(args...), optionally as a
+// programmatic dependent launch of the preceding kernel on s.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                      Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 cudaError_t launch_router(const uint16_t* x, const float* Wr, const float* bias, int T, int d, int E, int k,
                           int split, float* zpart, int* tickets, int32_t* idx, float* gate, cudaStream_t s);
 cudaError_t launch_router_topk(const float* logits, int T, int E, int k, int32_t* idx, float* gate, cudaStream_t s);
@@ -279,7 +304,7 @@ __host__ __device__ inline int tile_table_offset(int mat, int fmt, int n_seg) {
   return (mat * 3 + (fmt - 1)) * (n_seg + 1);
 }
 
-cudaError_t launch_schedule(const int32_t* idx, int T, int k, int E, int S, int bn, int mb3, int mb4,
+cudaError_t launch_schedule(bool pdl, const int32_t* idx, int T, int k, int E, int S, int bn, int mb3, int mb4,
                             const int32_t* seg_fmt, int32_t* counts, int32_t* offsets, int32_t* sorted_token,
                             int32_t* inv_pos, int32_t* seg_off, int32_t* seg_cnt, int32_t* tiles, int32_t* scratch,
                             cudaStream_t s);
@@ -287,14 +312,14 @@ size_t schedule_scratch_ints(int max_tokens, int E);
 
 bool gemm_bn_supported(int bn);
 
-cudaError_t launch_grouped_gemm(const GemmArgs& a, const CUtensorMap& act_map, int fmt, int bn, int num_sms,
+cudaError_t launch_grouped_gemm(bool pdl, const GemmArgs& a, const CUtensorMap& act_map, int fmt, int bn, int num_sms,
                                 cudaStream_t s);
 
 // xp[p] = x[sorted_token[p]] for p < P (activation rows in schedule order).
-cudaError_t launch_permute_rows(const uint16_t* x, const int32_t* sorted_token, int P, int d, uint16_t* xp,
+cudaError_t launch_permute_rows(bool pdl, const uint16_t* x, const int32_t* sorted_token, int P, int d, uint16_t* xp,
                                 cudaStream_t s);
 
-cudaError_t launch_combine(const uint16_t* Y, const float* gate, const int32_t* inv_pos, int T, int k, int S,
+cudaError_t launch_combine(bool pdl, const uint16_t* Y, const float* gate, const int32_t* inv_pos, int T, int k, int S,
                            int d, uint16_t* out, cudaStream_t s);
 
 cudaError_t launch_repack(int fmt, int mat, const void* w, const void* scale, int rows, int K, int I,

@@ -115,6 +115,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_fused_kernel(
   const int t0 = tt * RT, e0 = et * RE;
   const int slice = d / split, c_begin = sp * slice, nchunks = slice / RC;
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  pdl_wait();                                   // x may come from the previous kernel on the stream
 
   auto issue = [&](int chunk, int stage) {
     const int c0 = c_begin + chunk * RC;

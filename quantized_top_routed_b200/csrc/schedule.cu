@@ -45,6 +45,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int32_t s_fmt[kMaxE + kMaxShared];
   int32_t* hist = hist_in_smem ? hist_smem : hist_global;   // [C][E]: chunk counts, then chunk bases
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_wait();                                   // the router's indices are complete past this point
   const int C = (T + 31) / 32;
   const uint32_t lt_mask = (1u << lane) - 1u;
 
@@ -157,7 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 size_t schedule_scratch_ints(int max_tokens, int E) { return (size_t)((max_tokens + 31) / 32) * E; }
 
-cudaError_t launch_schedule(const int32_t* idx, int T, int k, int E, int S, int bn, int mb3, int mb4,
+cudaError_t launch_schedule(bool pdl, const int32_t* idx, int T, int k, int E, int S, int bn, int mb3, int mb4,
                             const int32_t* seg_fmt, int32_t* counts, int32_t* offsets, int32_t* sorted_token,
                             int32_t* inv_pos, int32_t* seg_off, int32_t* seg_cnt, int32_t* tiles, int32_t* scratch,
                             cudaStream_t s) {
@@ -169,9 +170,8 @@ cudaError_t launch_schedule(const int32_t* idx, int T, int k, int E, int S, int 
     cudaError_t e = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kHistSmemMax);
     if (e != cudaSuccess) return e;
   }
-  schedule_kernel<<<1, kThreads, dyn, s>>>(idx, T, k, E, S, bn, mb3, mb4, seg_fmt, counts, offsets, sorted_token,
-                                           inv_pos, seg_off, seg_cnt, tiles, scratch, in_smem);
-  return cudaGetLastError();
+  return launch_ex(schedule_kernel, dim3(1), dim3(kThreads), dyn, s, pdl, idx, T, k, E, S, bn, mb3, mb4, seg_fmt,
+                   counts, offsets, sorted_token, inv_pos, seg_off, seg_cnt, tiles, scratch, in_smem);
 }
 
 }  // namespace qmoe
