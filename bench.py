@@ -362,6 +362,14 @@ def traffic_from_profiles(L, kernel):
         return None
     with open(p) as f:
         d = json.load(f)
+    # counters taken on another version of the kernel say nothing about this one
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("gemm.cu", "qmoe_internal.cuh"):
+        with open(os.path.join(ROOT, "quantized_top_routed_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    if d.get("kernel_source_sha256") != h.hexdigest():
+        return None
     key = f"{L.name}:T={L.T}:{kernel}"
     v = d.get(key)
     return None if v is None else v.get("dram_bytes_per_launch")
@@ -444,7 +452,7 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-sweep", dest="sweep", action="store_false")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-tokens", type=int, default=16, help="tokens in the timed oracle sample")
+    ap.add_argument("--cpu-tokens", type=int, default=48, help="tokens in the timed oracle sample")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
