@@ -173,17 +173,17 @@ const char* qmoe_last_error(void);
  * T * E <= QMOE_ROUTE_STATIC_MAX_LOGITS; larger sizes are rejected with
  * QMOE_ERR_INVALID and nothing is enqueued.
  *
- * Scratch: the router's partial logits and its per-token-tile counters live
- * in one fixed library-global device array of QMOE_ROUTE_STATIC_SCRATCH_BYTES
- * bytes per device (no cudaMalloc, cudaFree or allocating library call is
- * made).  The counters are cleared with cudaMemsetAsync on `stream` before
- * each launch.  The array's address is looked up once per device on the
- * first call (cudaGetSymbolAddress, which may load the module), so make that
- * first call before any stream capture begins.  Because the scratch is
- * shared, calls whose work may overlap on the same GPU (different streams,
- * or different host threads) race and give wrong results: serialise them. */
+ * Scratch: the router's partial logits live in one fixed library-global
+ * device array of QMOE_ROUTE_STATIC_SCRATCH_BYTES bytes per device (no
+ * cudaMalloc, cudaFree or allocating library call is made; every scratch
+ * element read is first written by the same call, so nothing is cleared).
+ * The array's address is looked up once per device on the first call
+ * (cudaGetSymbolAddress, which may load the module), so make that first
+ * call before any stream capture begins.  Because the scratch is shared,
+ * calls whose work may overlap on the same GPU (different streams, or
+ * different host threads) race and give wrong results: serialise them. */
 #define QMOE_ROUTE_STATIC_MAX_LOGITS (1 << 20)
-#define QMOE_ROUTE_STATIC_SCRATCH_BYTES (4 * (1 << 20) + 4 * (1 << 15))
+#define QMOE_ROUTE_STATIC_SCRATCH_BYTES (4 * (1 << 20))
 qmoe_status qmoe_route_topk_noalloc(const uint16_t* x, const float* router_w, const float* router_bias,
                                     int32_t T, int32_t d, int32_t E, int32_t k, int32_t* topk_idx,
                                     float* topk_gate, void* stream);

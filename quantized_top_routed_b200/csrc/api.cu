@@ -99,7 +99,6 @@ struct qmoe_handle {
   CUtensorMap xp_map[kNumBn];            // permuted x rows (gate/up B operand), one per block width
   CUtensorMap h_map[kNumBn];             // H rows (down B operand), one per block width
   float *gates = nullptr, *zpart = nullptr;
-  int* tickets = nullptr;
   uint16_t *Xp = nullptr, *H = nullptr, *Y = nullptr, *x_stage = nullptr, *out_stage = nullptr;
   int* err = nullptr;
   int zpart_split_max = 1;
@@ -195,7 +194,7 @@ qmoe_status route_impl(qmoe_handle* h, const uint16_t* x, const float* logits, i
     if (x) {
       int split = router_split(T, c.d, c.E, h->num_sms);
       if (split > h->zpart_split_max) split = h->zpart_split_max;
-      QMOE_CUDA(launch_router(x, h->router_w, h->router_b, T, c.d, c.E, c.k, split, h->zpart, h->tickets, idx,
+      QMOE_CUDA(launch_router(x, h->router_w, h->router_b, T, c.d, c.E, c.k, split, h->zpart, idx,
                               gates, s),
                 "router launch");
     } else {
@@ -343,10 +342,6 @@ qmoe_status qmoe_create(const qmoe_config* cfg, const float* router_w, const flo
   if ((st = h->alloc(&h->out_stage, Tm * c.d, "out staging")) != QMOE_OK) return bail(st);
   if ((st = h->alloc(&h->err, 1, "error word")) != QMOE_OK) return bail(st);
   if (cudaMemset(h->err, 0, sizeof(int)) != cudaSuccess) return bail(cuda_fail(cudaGetLastError(), "memset"));
-  const int ntick = router_tickets(c.max_tokens);
-  if ((st = h->alloc(&h->tickets, (size_t)ntick, "router tickets")) != QMOE_OK) return bail(st);
-  if (cudaMemset(h->tickets, 0, sizeof(int) * ntick) != cudaSuccess)
-    return bail(cuda_fail(cudaGetLastError(), "memset"));
   cudaError_t se = cudaDeviceSynchronize();
   if (se != cudaSuccess) return bail(cuda_fail(se, "qmoe_create"));
   *out = h;
@@ -469,7 +464,7 @@ int32_t qmoe_launches_per_forward(const qmoe_handle* h, int32_t T) {
   if (!h) return 0;
   int fmts = 0;
   for (int f = 1; f <= 3; ++f) fmts += h->fmt_present[f] ? 1 : 0;
-  return 4 + 2 * fmts;  // router, schedule, row permutation, gate/up and down GEMM per format, combine
+  return 5 + 2 * fmts;  // router logits + top-k, schedule, row permutation, gate/up and down per format, combine
 }
 
 qmoe_status qmoe_destroy(qmoe_handle* h) {
@@ -483,14 +478,13 @@ qmoe_status qmoe_destroy(qmoe_handle* h) {
 }  // extern "C"
 
 // ---- routing without a handle and without allocation ------------------------
-// One fixed device array per device holds the router's partial logits and its
-// per-token-tile counters: counters first (one int per 32-token tile), then
-// the partial-logit slices.  Nothing here allocates device memory.
+// One fixed device array per device holds the router's partial logits (every
+// element that is read is written first by the same call, so nothing needs
+// clearing).  Nothing here allocates device memory.
 namespace {
 
-constexpr size_t kNoallocTickets = size_t(1) << 15;            // ints: covers T up to 2^20
 constexpr size_t kNoallocLogits = QMOE_ROUTE_STATIC_MAX_LOGITS;  // floats
-static_assert(QMOE_ROUTE_STATIC_SCRATCH_BYTES == 4 * (kNoallocLogits + kNoallocTickets), "scratch size");
+static_assert(QMOE_ROUTE_STATIC_SCRATCH_BYTES == 4 * kNoallocLogits, "scratch size");
 static __device__ __align__(256) unsigned char g_route_scratch[QMOE_ROUTE_STATIC_SCRATCH_BYTES];
 
 constexpr int kNoallocMaxDevices = 64;
@@ -537,14 +531,11 @@ qmoe_status qmoe_route_topk_noalloc(const uint16_t* x, const float* router_w, co
   int sms = 0;
   qmoe_status st = noalloc_scratch(&base, &sms);
   if (st != QMOE_OK) return st;
-  int* tickets = static_cast<int*>(base);
-  float* zpart = reinterpret_cast<float*>(static_cast<int*>(base) + kNoallocTickets);
+  float* zpart = static_cast<float*>(base);
   int split = router_split(T, d, E, sms);
   while (split > 1 && (long long)split * T * E > (long long)kNoallocLogits) split >>= 1;
-  const int ntick = router_tickets(T);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  QMOE_CUDA(cudaMemsetAsync(tickets, 0, sizeof(int) * (size_t)ntick, s), "clear routing counters");
-  QMOE_CUDA(launch_router(x, router_w, router_bias, T, d, E, k, split, zpart, tickets, topk_idx, topk_gate, s),
+  QMOE_CUDA(launch_router(x, router_w, router_bias, T, d, E, k, split, zpart, topk_idx, topk_gate, s),
             "router launch");
   return QMOE_OK;
 }

@@ -292,10 +292,9 @@ cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem
 }
 
 cudaError_t launch_router(const uint16_t* x, const float* Wr, const float* bias, int T, int d, int E, int k,
-                          int split, float* zpart, int* tickets, int32_t* idx, float* gate, cudaStream_t s);
+                          int split, float* zpart, int32_t* idx, float* gate, cudaStream_t s);
 cudaError_t launch_router_topk(const float* logits, int T, int E, int k, int32_t* idx, float* gate, cudaStream_t s);
 int router_split(int T, int d, int E, int num_sms);
-int router_tickets(int max_tokens);
 
 // Tile tables written by the schedule kernel: for matrix m (0 gate/up, 1
 // down) and weight format f (1..3), tiles + tile_table_offset(m, f, n_seg)

@@ -5,14 +5,13 @@
 // top-k routing; "FineRMoE", Sparse Sum Layer: softmax probabilities as
 // mixing weights.)
 //
-// From activations (one launch): router_fused_kernel computes a 32-token x
-// 32-expert tile of fp32 logits over one slice of d (d is split so the grid
+// From activations (two launches): router_logits_kernel computes a 32-token
+// x 32-expert tile of fp32 logits over one slice of d (d is split so the grid
 // covers the SMs when T is small), streaming x and Wr through a 3-stage
-// cp.async ring.  Each CTA writes its partial sums, then takes a ticket for
-// its token tile; the CTA that completes the tile sums the partials of all
-// slices in a fixed order (so the logits are deterministic) and runs the
-// warp-per-token top-k for the tile's 32 tokens, then resets the ticket.
-// From supplied logits: router_topk_kernel alone, one warp per token.
+// cp.async ring, and writes its partial sums; router_topk_kernel then runs
+// one warp per token, which sums the slices in a fixed order (so the logits
+// are deterministic), adds the bias and takes the top-k.  From supplied
+// logits: router_topk_kernel alone, with one slice.
 #include "qmoe_internal.cuh"
 
 #include <math.h>
@@ -28,7 +27,7 @@ constexpr int XS = RC + 8;      // bf16 row stride of the x stage (bank shift of
 constexpr int WS = RC + 4;      // fp32 row stride of the Wr stage
 constexpr int kRouterThreads = 256;
 constexpr int kSmemPipe = NST * (RT * XS * 2 + RE * WS * 4);
-constexpr int kSmemRouter = kSmemPipe > RT * kMaxE * 4 ? kSmemPipe : RT * kMaxE * 4;
+constexpr int kSmemRouter = kSmemPipe;
 
 // Warp arg-max over (value, index): larger value wins, lower index on ties.
 __device__ __forceinline__ void warp_argmax(float& v, int& e) {
@@ -102,15 +101,12 @@ __device__ __forceinline__ void cp16(uint32_t dst, const void* src, uint32_t n) 
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
 }
 
-template <int EPL>
-__global__ void __launch_bounds__(kRouterThreads) router_fused_kernel(
-    const uint16_t* __restrict__ x, const float* __restrict__ Wr, const float* __restrict__ bias, int T, int d,
-    int E, int k, int split, float* __restrict__ zpart, int* __restrict__ tickets, int32_t* __restrict__ idx,
-    float* __restrict__ gate) {
+__global__ void __launch_bounds__(kRouterThreads) router_logits_kernel(const uint16_t* __restrict__ x,
+                                                                      const float* __restrict__ Wr, int T, int d,
+                                                                      int E, int split, float* __restrict__ zpart) {
   extern __shared__ __align__(16) uint8_t rsm[];
   uint16_t* xs = reinterpret_cast<uint16_t*>(rsm);                          // [NST][RT][XS]
   float* ws = reinterpret_cast<float*>(rsm + NST * RT * XS * 2);            // [NST][RE][WS]
-  __shared__ int s_last;
   const int tt = blockIdx.x, et = blockIdx.y, sp = blockIdx.z;
   const int t0 = tt * RT, e0 = et * RE;
   const int slice = d / split, c_begin = sp * slice, nchunks = slice / RC;
@@ -178,69 +174,36 @@ __global__ void __launch_bounds__(kRouterThreads) router_fused_kernel(
   if (ta < T && eb < E) zp[(size_t)ta * E + eb] = acc01;
   if (tb < T && ea < E) zp[(size_t)tb * E + ea] = acc10;
   if (tb < T && eb < E) zp[(size_t)tb * E + eb] = acc11;
-
-  // ---- the CTA that completes a token tile runs its top-k ----------------
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const int need = gridDim.y * gridDim.z;
-    const int ticket = atomicAdd(&tickets[tt], 1);
-    s_last = ticket == need - 1;
-    if (s_last) tickets[tt] = 0;  // ready for the next call
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  // Sum the slices of this tile's logits into shared memory (coalesced,
-  // every load in flight at once), then one warp per token runs the top-k.
-  float* zs = reinterpret_cast<float*>(rsm);                   // [RT][E], reuses the pipeline buffers
-  const int rows = min(RT, T - t0);
-  const int nel = rows * E;                                     // the tile's rows are contiguous in zpart
-  constexpr int kPer = RT * 32 * EPL / kRouterThreads;          // elements per thread (E <= 32 * EPL)
-  float acc[kPer];
-#pragma unroll
-  for (int m = 0; m < kPer; ++m) acc[m] = 0.f;
-  for (int s2 = 0; s2 < split; ++s2) {                          // one round trip per slice
-    const float* zp2 = zpart + ((size_t)s2 * T + t0) * E;
-#pragma unroll
-    for (int m = 0; m < kPer; ++m) {
-      const int v = tid + m * kRouterThreads;
-      if (v < nel) acc[m] += __ldcg(zp2 + v);
-    }
-  }
-#pragma unroll
-  for (int m = 0; m < kPer; ++m) {
-    const int v = tid + m * kRouterThreads;
-    if (v < nel) zs[v] = bias ? acc[m] + bias[v % E] : acc[m];
-  }
-  __syncthreads();
-  const int warp = tid >> 5, lane = tid & 31;
-  for (int r = warp; r < rows; r += kRouterThreads / 32) {
-    const int t = t0 + r;
-    auto logit = [&](int e) { return zs[r * E + e]; };
-    topk_token<EPL>(logit, E, k, lane, idx + (size_t)t * k, gate + (size_t)t * k);
-  }
 }
 
+// One warp per token: logit(e) = sum over slices s (in order) of zpart[s][t][e],
+// plus the bias, then softmax, top-k and renormalisation.
 template <int EPL>
-__global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
+__global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ zpart, int split,
+                                                          const float* __restrict__ bias, int T, int E, int k,
                                                           int32_t* __restrict__ idx, float* __restrict__ gate) {
+  pdl_wait();
   const int t = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
-  auto logit = [&](int e) { return logits[(size_t)t * E + e]; };
+  auto logit = [&](int e) {
+    float acc = 0.f;
+    for (int s2 = 0; s2 < split; ++s2) acc += __ldcg(zpart + ((size_t)s2 * T + t) * E + e);
+    return bias ? acc + bias[e] : acc;
+  };
   topk_token<EPL>(logit, E, k, lane, idx + (size_t)t * k, gate + (size_t)t * k);
 }
 
-template <int EPL>
-cudaError_t launch_fused(const uint16_t* x, const float* Wr, const float* bias, int T, int d, int E, int k, int split,
-                         float* zpart, int* tickets, int32_t* idx, float* gate, cudaStream_t s) {
-  auto kern = router_fused_kernel<EPL>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemRouter);
-  if (e != cudaSuccess) return e;
-  dim3 grid((T + RT - 1) / RT, (E + RE - 1) / RE, split);
-  kern<<<grid, kRouterThreads, kSmemRouter, s>>>(x, Wr, bias, T, d, E, k, split, zpart, tickets, idx, gate);
-  return cudaGetLastError();
+cudaError_t launch_topk(const float* zpart, int split, const float* bias, int T, int E, int k, int32_t* idx,
+                        float* gate, cudaStream_t s) {
+  const dim3 blocks((T + 7) / 8), threads(256);
+  switch ((E + 31) / 32) {
+    case 1: return launch_ex(router_topk_kernel<1>, blocks, threads, 0, s, false, zpart, split, bias, T, E, k, idx, gate);
+    case 2: return launch_ex(router_topk_kernel<2>, blocks, threads, 0, s, false, zpart, split, bias, T, E, k, idx, gate);
+    case 3:
+    case 4: return launch_ex(router_topk_kernel<4>, blocks, threads, 0, s, false, zpart, split, bias, T, E, k, idx, gate);
+    default: return launch_ex(router_topk_kernel<8>, blocks, threads, 0, s, false, zpart, split, bias, T, E, k, idx, gate);
+  }
 }
 
 }  // namespace
@@ -254,31 +217,19 @@ int router_split(int T, int d, int E, int num_sms) {
   return split;
 }
 
-int router_tickets(int max_tokens) { return (max_tokens + RT - 1) / RT; }
-
 cudaError_t launch_router(const uint16_t* x, const float* Wr, const float* bias, int T, int d, int E, int k, int split,
-                          float* zpart, int* tickets, int32_t* idx, float* gate, cudaStream_t s) {
-  const int epl = (E + 31) / 32;
-  switch (epl) {
-    case 1: return launch_fused<1>(x, Wr, bias, T, d, E, k, split, zpart, tickets, idx, gate, s);
-    case 2: return launch_fused<2>(x, Wr, bias, T, d, E, k, split, zpart, tickets, idx, gate, s);
-    case 3:
-    case 4: return launch_fused<4>(x, Wr, bias, T, d, E, k, split, zpart, tickets, idx, gate, s);
-    default: return launch_fused<8>(x, Wr, bias, T, d, E, k, split, zpart, tickets, idx, gate, s);
-  }
+                          float* zpart, int32_t* idx, float* gate, cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(router_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemRouter);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((T + RT - 1) / RT, (E + RE - 1) / RE, split);
+  e = launch_ex(router_logits_kernel, grid, dim3(kRouterThreads), kSmemRouter, s, false, x, Wr, T, d, E, split,
+                zpart);
+  if (e != cudaSuccess) return e;
+  return launch_topk(zpart, split, bias, T, E, k, idx, gate, s);
 }
 
 cudaError_t launch_router_topk(const float* logits, int T, int E, int k, int32_t* idx, float* gate, cudaStream_t s) {
-  const int blocks = (T + 7) / 8;
-  const int epl = (E + 31) / 32;
-  switch (epl) {
-    case 1: router_topk_kernel<1><<<blocks, 256, 0, s>>>(logits, T, E, k, idx, gate); break;
-    case 2: router_topk_kernel<2><<<blocks, 256, 0, s>>>(logits, T, E, k, idx, gate); break;
-    case 3:
-    case 4: router_topk_kernel<4><<<blocks, 256, 0, s>>>(logits, T, E, k, idx, gate); break;
-    default: router_topk_kernel<8><<<blocks, 256, 0, s>>>(logits, T, E, k, idx, gate); break;
-  }
-  return cudaGetLastError();
+  return launch_topk(logits, 1, nullptr, T, E, k, idx, gate, s);
 }
 
 }  // namespace qmoe
