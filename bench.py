@@ -93,6 +93,13 @@ def workload_desc(L) -> str:
             f"weights={'+'.join(fmts)}" + (" zipf-bias" if L.router_b is not None else ""))
 
 
+def compute_dtype(L) -> str:
+    """MMA input type: a layer whose experts are all FP8 computes in fp16
+    (exact e4m3 -> fp16 conversion), any other layer in bf16."""
+    from quantized_top_routed_b200 import synth
+    return "f16" if all(ex.fmt == synth.FMT_FP8 for ex in L.experts) else "bf16"
+
+
 def gate_up_bytes(L, touched) -> int:
     """Algorithmic HBM bytes of one gate/up GEMM launch: the codes and scales of
     every touched expert's W13 (and always-on shared experts), the token rows
@@ -293,7 +300,7 @@ def run_ours(args):
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, shapes of the workload)",
+        "vs_baseline": None, "dtype": compute_dtype(L), "data": "synthetic (seeded, shapes of the workload)",
         "config": {"workload": workload_desc(L), "T": T, "global_batch": world * T, "parallelism": f"replicas x{world}",
                    "l2": "flushed between timed steps (256 MB write)", "touched_experts": len(touched)},
         "layer": {"bytes": layer_bytes(L, touched), "flops": layer_flops(L),

@@ -96,6 +96,7 @@ struct qmoe_handle {
   int32_t *idx = nullptr, *inv_pos = nullptr, *counts = nullptr, *offsets = nullptr, *sorted_token = nullptr;
   int32_t *seg_off = nullptr, *seg_cnt = nullptr, *tiles = nullptr, *seg_fmt = nullptr, *sched_scratch = nullptr;
   bool fmt_present[4] = {false, false, false, false};
+  bool mma_f16 = false;                  // all experts FP8: x rows, H and the MMAs in fp16
   CUtensorMap xp_map[kNumBn];            // permuted x rows (gate/up B operand), one per block width
   CUtensorMap h_map[kNumBn];             // H rows (down B operand), one per block width
   float *gates = nullptr, *zpart = nullptr;
@@ -276,6 +277,12 @@ qmoe_status qmoe_create(const qmoe_config* cfg, const float* router_w, const flo
       return bail(cuda_fail(cudaGetLastError(), "copy router_b"));
   }
 
+  // A layer whose experts are all FP8 computes in fp16: e4m3 codes convert to
+  // fp16 exactly with one instruction per pair, so x rows and H are fp16 too.
+  // Any other mix computes in bf16.
+  h->mma_f16 = true;
+  for (int e = 0; e < nexp; ++e) h->mma_f16 = h->mma_f16 && experts[e].fmt == QMOE_W_FP8_E4M3_PC;
+
   // experts: repack both matrices of each expert into handle-owned tiles
   std::vector<ExpertDev> host_desc(nexp);
   for (int e = 0; e < nexp; ++e) {
@@ -294,7 +301,8 @@ qmoe_status qmoe_create(const qmoe_config* cfg, const float* router_w, const flo
       if ((st = h->alloc(&wdst, tiles * stage_bytes(x.fmt), "expert weights")) != QMOE_OK) return bail(st);
       if (x.fmt != QMOE_W_INT4_G128)
         if ((st = h->alloc(&sdst, (size_t)rows[m], "expert scales")) != QMOE_OK) return bail(st);
-      cudaError_t e2 = launch_repack(x.fmt, m, ws[m], ss[m], rows[m], Ks[m], c.I, wdst, sdst, 0);
+      cudaError_t e2 = launch_repack(h->mma_f16 ? kFmtFp8F16 : x.fmt, m, ws[m], ss[m], rows[m], Ks[m], c.I, wdst,
+                                     sdst, 0);
       if (e2 != cudaSuccess) return bail(cuda_fail(e2, "repack launch"));
       dv.w[m] = wdst;
       dv.spc[m] = sdst;
@@ -377,7 +385,8 @@ qmoe_status qmoe_forward(qmoe_handle* h, const uint16_t* x, int32_t T, uint16_t*
   {
     // x rows in schedule order (the permutation half of stage 2)
     StageTimer tm(h, s, QMOE_STAGE_SCHEDULE);
-    QMOE_CUDA(launch_permute_rows(kUsePdl, x, h->sorted_token, T * (c.k + c.n_shared), c.d, h->Xp, s), "permute launch");
+    QMOE_CUDA(launch_permute_rows(kUsePdl, x, h->sorted_token, T * (c.k + c.n_shared), c.d, h->Xp, h->mma_f16, s),
+              "permute launch");
   }
   GemmArgs g{};
   g.experts = h->d_experts;
@@ -397,7 +406,8 @@ qmoe_status qmoe_forward(qmoe_handle* h, const uint16_t* x, int32_t T, uint16_t*
     for (int fmt = 1; fmt <= 3; ++fmt) {   // one launch per weight format present
       if (!h->fmt_present[fmt]) continue;
       g.tile_off = h->tiles + tile_table_offset(mat, fmt, g.n_seg);
-      QMOE_CUDA(launch_grouped_gemm(kUsePdl, g, mat == 0 ? h->xp_map[bn_index(bn)] : h->h_map[bn_index(bn)], fmt, bn,
+      const int kfmt = h->mma_f16 ? kFmtFp8F16 : fmt;
+      QMOE_CUDA(launch_grouped_gemm(kUsePdl, g, mat == 0 ? h->xp_map[bn_index(bn)] : h->h_map[bn_index(bn)], kfmt, bn,
                                     h->num_sms, s),
                 mat == 0 ? "gate/up GEMM launch" : "down GEMM launch");
     }

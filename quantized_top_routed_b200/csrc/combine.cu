@@ -9,6 +9,8 @@
 //
 // Each thread moves one 16-byte vector (8 bf16) of one token, so every Y row
 // and the output row are read and written with coalesced 16-byte accesses.
+#include <cuda_fp16.h>
+
 #include "qmoe_internal.cuh"
 
 namespace qmoe {
@@ -70,23 +72,32 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
 // 16-byte vector, so each row is read and written with coalesced accesses.
 __global__ void __launch_bounds__(256) permute_rows_kernel(const uint16_t* __restrict__ x,
                                                            const int32_t* __restrict__ sorted_token, int P, int d,
-                                                           uint16_t* __restrict__ xp) {
+                                                           uint16_t* __restrict__ xp, int to_f16) {
   pdl_wait();                                   // the schedule's permutation is complete past this point
   const int nvec = d >> 3;
   const long long gv = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (gv >= (long long)P * nvec) return;
   const int p = (int)(gv / nvec), v = (int)(gv - (long long)p * nvec);
   const int t = __ldg(sorted_token + p);
-  reinterpret_cast<uint4*>(xp + (size_t)p * d)[v] = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d) + v);
+  uint4 q = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d) + v);
+  if (to_f16) {                                 // bf16 -> fp16 (exact inside the fp16 range)
+    uint32_t* w = reinterpret_cast<uint32_t*>(&q);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __half2 h = __floats2half2_rn(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+      w[i] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+  }
+  reinterpret_cast<uint4*>(xp + (size_t)p * d)[v] = q;
 }
 
 }  // namespace
 
 cudaError_t launch_permute_rows(bool pdl, const uint16_t* x, const int32_t* sorted_token, int P, int d, uint16_t* xp,
-                                cudaStream_t s) {
+                                bool to_f16, cudaStream_t s) {
   const long long n = (long long)P * (d >> 3);
   return launch_ex(permute_rows_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, pdl, x, sorted_token, P,
-                   d, xp);
+                   d, xp, to_f16 ? 1 : 0);
 }
 
 cudaError_t launch_combine(bool pdl, const uint16_t* Y, const float* gate, const int32_t* inv_pos, int T, int k, int S, int d,

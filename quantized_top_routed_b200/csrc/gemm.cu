@@ -46,6 +46,7 @@
 // Every wait is bounded: a role that waits ~1 s raises an abort flag, all
 // roles drain what they issued, TMEM is freed and the error word is set.
 #include <cuda.h>
+#include <cuda_fp16.h>
 
 #include <type_traits>
 
@@ -167,7 +168,18 @@ __device__ __forceinline__ void deq_fp8_word(uint32_t w, uint32_t* o) {
   o[1] = bf2_mul(hi, 0x7B807B80u);
 }
 
-// This thread's 16-byte chunks (K order) -> kHalf / 2 bf16 pairs.
+// 4 e4m3 codes (natural K order) -> 2 fp16 pairs (exact), one hardware
+// conversion per pair of codes.
+__device__ __forceinline__ void deq_fp8_f16_word(uint32_t w, uint32_t* o) {
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "mov.b32 {lo, hi}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, lo;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
+      : "=r"(o[0]), "=r"(o[1])
+      : "r"(w));
+}
+
+// This thread's 16-byte chunks (K order) -> kHalf / 2 bf16 (or fp16) pairs.
 template <int FMT>
 __device__ __forceinline__ void dequant_slice(const uint4 (&w)[FmtCfg<FMT>::NC], uint32_t sbits, uint32_t* av) {
 #pragma unroll
@@ -178,6 +190,11 @@ __device__ __forceinline__ void dequant_slice(const uint4 (&w)[FmtCfg<FMT>::NC],
       deq_int4_word(w[c].y, s2, &av[16 * c + 4]);
       deq_int4_word(w[c].z, s2, &av[16 * c + 8]);
       deq_int4_word(w[c].w, s2, &av[16 * c + 12]);
+    } else if constexpr (FMT == kFmtFp8F16) {
+      deq_fp8_f16_word(w[c].x, &av[8 * c + 0]);
+      deq_fp8_f16_word(w[c].y, &av[8 * c + 2]);
+      deq_fp8_f16_word(w[c].z, &av[8 * c + 4]);
+      deq_fp8_f16_word(w[c].w, &av[8 * c + 6]);
     } else if constexpr (FMT == QMOE_W_FP8_E4M3_PC) {
       deq_fp8_word(w[c].x, &av[8 * c + 0]);
       deq_fp8_word(w[c].y, &av[8 * c + 2]);
@@ -197,6 +214,10 @@ __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)
 __device__ __forceinline__ uint16_t f2bf(float f) {
   const __nv_bfloat16 b = __float2bfloat16_rn(f);
   return *reinterpret_cast<const uint16_t*>(&b);
+}
+__device__ __forceinline__ uint16_t f2h(float f) {
+  const __half h = __float2half_rn(f);
+  return *reinterpret_cast<const uint16_t*>(&h);
 }
 
 // TMA: a box of 64 bf16 columns x BN rows of a row-major matrix into
@@ -373,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = mbar_wait(&acc_empty[2 * j + b], ((q >> 1) & 1) ^ 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t idesc = idesc_bf16_m128(max(16, (t.nvalid + 15) & ~15));
+        const uint32_t idesc = idesc_bf16_m128(max(16, (t.nvalid + 15) & ~15), FMT == kFmtFp8F16);
         const uint32_t d_tmem = tmem_base + (uint32_t)((2 * j + b) * BN);
         const int u0 = q * KS;                 // super-stage index of this group's first K stage
         uint32_t s = (uint32_t)(u0 % C::SP), ph = (uint32_t)((u0 / C::SP) & 1);
@@ -514,7 +535,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 16; ++i) {
               const float f = __uint_as_float(v[i]) * scale;
               const float o = __shfl_xor_sync(0xffffffffu, f, 1);   // up value of the same index
-              if ((lane & 1) == 0) stg[(c0 + i) * WCOLS + (lane >> 1)] = f2bf(silu_f(f) * o);
+              if ((lane & 1) == 0) {
+                const float hv = silu_f(f) * o;   // H is fp16 in the fp16 MMA mode, else bf16
+                stg[(c0 + i) * WCOLS + (lane >> 1)] = FMT == kFmtFp8F16 ? f2h(hv) : f2bf(hv);
+              }
             }
           } else {
 #pragma unroll
@@ -560,6 +584,7 @@ cudaError_t launch_fmt(bool pdl, const GemmArgs& a, const CUtensorMap& map, int 
     case QMOE_W_INT4_G128: return launch_one<BN, MAT, QMOE_W_INT4_G128>(pdl, a, map, num_sms, s);
     case QMOE_W_FP8_E4M3_PC: return launch_one<BN, MAT, QMOE_W_FP8_E4M3_PC>(pdl, a, map, num_sms, s);
     case QMOE_W_INT8_PC: return launch_one<BN, MAT, QMOE_W_INT8_PC>(pdl, a, map, num_sms, s);
+    case kFmtFp8F16: return launch_one<BN, MAT, kFmtFp8F16>(pdl, a, map, num_sms, s);
     default: return cudaErrorInvalidValue;
   }
 }

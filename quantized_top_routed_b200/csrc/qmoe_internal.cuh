@@ -28,6 +28,12 @@ struct ExpertDev {
   int32_t pad;
 };
 
+// Internal code of FP8 e4m3 weights when the whole layer computes in fp16:
+// the codes convert to fp16 with one hardware instruction per pair, and the
+// activations and H are then fp16 too (an MMA takes one input type).  Same
+// tile layout as QMOE_W_FP8_E4M3_PC except the byte order inside a word.
+constexpr int kFmtFp8F16 = 4;
+
 // Bytes of one repacked (128 rows x 128 K) tile.  INT4 tiles carry their
 // 128 bf16 group scales after the codes.
 __host__ __device__ inline int stage_bytes(int fmt) {
@@ -252,10 +258,10 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
 }
 
 // Instruction descriptor, kind::f16: bf16 A and B (both K-major), fp32 D, M = 128.
-__host__ __device__ constexpr uint32_t idesc_bf16_m128(int n) {
+__host__ __device__ constexpr uint32_t idesc_bf16_m128(int n, bool f16 = false) {
   return (1u << 4)                          // D format: f32
-         | (1u << 7)                        // A format: bf16
-         | (1u << 10)                       // B format: bf16
+         | ((f16 ? 0u : 1u) << 7)           // A format: bf16 (1) or f16 (0)
+         | ((f16 ? 0u : 1u) << 10)          // B format: the same type as A
          | ((uint32_t)(n >> 3) << 17)       // N / 8
          | ((uint32_t)(128 >> 4) << 24);    // M / 16
 }
@@ -315,8 +321,9 @@ cudaError_t launch_grouped_gemm(bool pdl, const GemmArgs& a, const CUtensorMap& 
                                 cudaStream_t s);
 
 // xp[p] = x[sorted_token[p]] for p < P (activation rows in schedule order).
+// to_f16: write the rows as fp16 (the fp16 MMA mode) instead of copying bf16.
 cudaError_t launch_permute_rows(bool pdl, const uint16_t* x, const int32_t* sorted_token, int P, int d, uint16_t* xp,
-                                cudaStream_t s);
+                                bool to_f16, cudaStream_t s);
 
 cudaError_t launch_combine(bool pdl, const uint16_t* Y, const float* gate, const int32_t* inv_pos, int T, int k, int S,
                            int d, uint16_t* out, cudaStream_t s);

@@ -14,7 +14,8 @@
 // Byte order inside a chunk (chosen for the in-register dequantisation):
 //   INT8 / FP8 (16 K elements per chunk): each 32-bit word holds K elements
 //     (k0, k2, k1, k3) in bytes 0..3, so bytes {0,2} and {1,3} expand to
-//     bf16 pairs (k0,k1), (k2,k3).
+//     bf16 pairs (k0,k1), (k2,k3); FP8 for the fp16 MMA mode keeps the
+//     natural order (k0, k1, k2, k3), one hardware conversion per 16 bits.
 //   INT4 (32 K elements per chunk): each 32-bit word holds 8 K elements as
 //     biased nibbles (q + 8); nibble n < 4 is element 2n, nibble n >= 4 is
 //     element 2(n-4)+1, so (w >> 4j) & 0x000F000F yields the pair (2j, 2j+1).
@@ -69,7 +70,9 @@ __global__ void repack_kernel(int fmt, int mat, const uint8_t* __restrict__ w, c
       uint32_t words[4];
       for (int m = 0; m < 4; ++m) {
         const uint8_t* p = s + 16 * c + 4 * m;
-        words[m] = (uint32_t)p[0] | ((uint32_t)p[2] << 8) | ((uint32_t)p[1] << 16) | ((uint32_t)p[3] << 24);
+        words[m] = fmt == kFmtFp8F16
+                       ? ((uint32_t)p[0] | ((uint32_t)p[1] << 8) | ((uint32_t)p[2] << 16) | ((uint32_t)p[3] << 24))
+                       : ((uint32_t)p[0] | ((uint32_t)p[2] << 8) | ((uint32_t)p[1] << 16) | ((uint32_t)p[3] << 24));
       }
       uint4* o = reinterpret_cast<uint4*>(tile + c * 2048 + r * 16);
       *o = make_uint4(words[0], words[1], words[2], words[3]);

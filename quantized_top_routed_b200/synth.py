@@ -199,6 +199,8 @@ def zipf_bias(E: int, s: float, seed: int = 0) -> np.ndarray:
 def expert_format(cfg: dict, e: int) -> int:
     if cfg["fmt"] == "mixed":
         return FMT_INT8 if e < cfg["E"] // 2 else FMT_INT4
+    if cfg["fmt"] == "mixed_fp8":            # FP8 beside INT4: the layer computes in bf16
+        return FMT_FP8 if e < cfg["E"] // 2 else FMT_INT4
     return cfg["fmt"]
 
 

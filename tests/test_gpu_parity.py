@@ -195,6 +195,7 @@ def test_mixed_precision_full_size_sampled():
     dict(name="mixed", T=777, d=384, I=256, E=8, k=4, zipf=1.0),           # INT8 / INT4 mixed, skew
     dict(name="tiny", T=1000, d=256, I=512, E=8, k=2),                     # INT8, BN=128 tiles
     dict(name="decode", T=200, d=512, I=256, E=32, k=8),                   # INT4, BN=64
+    dict(name="mixed", T=333, d=256, I=256, E=8, k=2, fmt="mixed_fp8"),    # FP8 beside INT4 (bf16 MMAs)
 ])
 def test_multi_tile_ragged(kw):
     kw = dict(kw)
