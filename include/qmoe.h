@@ -107,7 +107,12 @@ typedef struct qmoe_handle qmoe_handle;
  * The weights are copied and re-laid-out into memory the handle owns, so
  * the caller may free its buffers once this returns; the workspace for
  * max_tokens is allocated here as well.  Synchronises the current device.
- * On success *out receives the handle; on failure *out is set to NULL. */
+ * On success *out receives the handle; on failure *out is set to NULL.
+ * Compute type: a layer whose experts are all FP8 e4m3 runs its GEMMs on
+ * fp16 inputs (the codes, x and the intermediate H convert to fp16 with at
+ * least bf16's precision), so its activations and H must stay inside the
+ * fp16 range (|v| < 65504); every other layer runs on bf16 inputs.  Both
+ * accumulate in fp32. */
 qmoe_status qmoe_create(const qmoe_config* cfg, const float* router_w, const float* router_bias,
                         const qmoe_expert* experts, qmoe_handle** out);
 
