@@ -87,6 +87,44 @@ def test_margin():
 
 
 # ---------------------------------------------------------------------------
+# router logits with a bias
+# ---------------------------------------------------------------------------
+def test_router_logits_with_bias_hand_case(golden_dir):
+    """Hand-worked logits, selection and gates with a non-zero bias and E != d."""
+    g = _load(golden_dir, "router_bias.json")
+    layer = _layer(g["x"], [], E=g["E"], k=g["k"], I=1, router_w=g["router_w"],
+                   router_b=np.asarray(g["router_b"], np.float32))
+    r = O.route(layer)
+    np.testing.assert_array_equal(r["logits"], g["logits"])
+    np.testing.assert_array_equal(r["idx"], g["idx"])
+    np.testing.assert_allclose(r["gates"], g["gates"], rtol=1e-15, atol=0)
+
+
+def test_router_logits_library_cross_check():
+    """z = x Wr^T + b against torch's float64 linear layer on random inputs."""
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(5)
+    T, d, E = 37, 96, 11
+    x_bits = synth.f32_to_bf16_bits(rng.standard_normal((T, d)).astype(np.float32))
+    w = rng.standard_normal((E, d)).astype(np.float32)
+    b = rng.standard_normal(E).astype(np.float32)
+    x64 = torch.from_numpy(synth.bf16_bits_as_f32(x_bits).astype(np.float64))
+    ref = torch.nn.functional.linear(x64, torch.from_numpy(w.astype(np.float64)),
+                                     torch.from_numpy(b.astype(np.float64))).numpy()
+    np.testing.assert_allclose(O.router_logits(x_bits, w, b), ref, rtol=1e-13, atol=1e-13)
+    ref0 = torch.nn.functional.linear(x64, torch.from_numpy(w.astype(np.float64))).numpy()
+    np.testing.assert_allclose(O.router_logits(x_bits, w, None), ref0, rtol=1e-13, atol=1e-13)
+
+
+def test_rel_l2_hand_value(golden_dir):
+    c = _load(golden_dir, "router_bias.json")["rel_l2_case"]
+    assert abs(O.rel_l2(c["a"], c["b"]) - c["value"]) < 1e-15
+    assert O.rel_l2(c["b"], c["b"]) == 0.0
+    # a second case: ||(0, 3, 4)|| / ||(0, 0, 10)|| = 5 / 10
+    assert abs(O.rel_l2([0.0, 3.0, 14.0], [0.0, 0.0, 10.0]) - 0.5) < 1e-15
+
+
+# ---------------------------------------------------------------------------
 # gates
 # ---------------------------------------------------------------------------
 def test_gates_sum_to_one_and_match_softmax_over_selected():
@@ -286,11 +324,11 @@ def test_from_logits_mode_uses_supplied_logits():
 # ---------------------------------------------------------------------------
 def _pins_pass(golden_dir):
     checks = [test_hand_expert_ffn, test_hand_routed_layer, test_routing_flip_worked_example,
-              test_e4m3_decode_golden]
+              test_e4m3_decode_golden, test_router_logits_with_bias_hand_case, test_rel_l2_hand_value]
     for chk in checks:
         try:
             chk(golden_dir)
-        except AssertionError:
+        except (AssertionError, ValueError):
             return False
     try:
         test_topk_ties_go_to_lower_index()
@@ -300,7 +338,8 @@ def _pins_pass(golden_dir):
         test_int4_pack_roundtrip_and_group_scales()
         test_shared_expert_adds_with_weight_one()
         test_dequant_int8_closed_form()
-    except AssertionError:
+        test_router_logits_library_cross_check()
+    except (AssertionError, ValueError):
         return False
     return True
 
@@ -322,6 +361,16 @@ MUTATIONS = {
     "int4_nibbles_swapped": ("unpack_int4", lambda p, K: O.__dict__["_orig_unpack_int4"](
         ((np.asarray(p, np.uint8) >> 4) | (np.asarray(p, np.uint8) << 4)).astype(np.uint8), K)),
     "schedule_tokens_descending": ("schedule", lambda idx, E: O.__dict__["_orig_schedule"](idx[::-1], E)),
+    "router_bias_dropped": ("router_logits", lambda x, w, b: O.__dict__["_orig_router_logits"](x, w, None)),
+    "router_bias_negated": ("router_logits", lambda x, w, b: O.__dict__["_orig_router_logits"](
+        x, w, None if b is None else -np.asarray(b, np.float32))),
+    "router_product_negated": ("router_logits", lambda x, w, b: O.__dict__["_orig_router_logits"](
+        x, -np.asarray(w, np.float32), b)),
+    "router_x_read_as_low_half": ("bf16_to_f64", lambda bits: (np.asarray(bits, np.uint16).astype(np.uint32))
+                                  .view(np.float32).astype(np.float64)),
+    "rel_l2_without_sqrt": ("rel_l2", lambda a, b: float(((np.asarray(a, np.float64) - np.asarray(b, np.float64)) ** 2)
+                                                        .sum()) / max(float((np.asarray(b, np.float64) ** 2).sum()), 1e-300)),
+    "rel_l2_relative_to_a": ("rel_l2", lambda a, b: O.__dict__["_orig_rel_l2"](b, a)),
 }
 
 
