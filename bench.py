@@ -2,17 +2,22 @@
 
 One step = one qmoe_forward (router, schedule, gate/up GEMM, down GEMM,
 combine) over one batch of seeded synthetic tokens already resident in HBM.
-Default workload: the decode-shaped layer (d=2048, E=128, top-8, I=768, INT4
+Headline workload: the decode-shaped layer (d=2048, E=128, top-8, I=768, INT4
 group-128 weights) at T=256 tokens, the largest of its token sweep; the
-other sweep points are reported under "sweep".  L2 (126 MB) is flushed by
+other sweep points are reported under "sweep".  On one GPU the same run then
+measures the prefill (T=8192, FP8), fine-grained + shared (T=4096, INT4,
+Zipf 1.2) and mixed-precision (T=16384, INT8/INT4, Zipf 1.0) layers, each
+under "configs" with its own roofline, warm-L2 companion, host-buffer e2e,
+realised expert load and CPU-oracle baseline.  L2 (126 MB) is flushed by
 writing a 256 MB buffer between timed steps, outside each step's events.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--T T]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--T T] [--also NAME ...]
   python bench.py --impl reference ...   # the fp64 CPU oracle on the same workload
 
 Multi-GPU (torchrun, one rank per GPU): the layer does not shard; every rank
 runs an independent replica on its own batch (weak scaling, no collective on
 the data path).  Timing is the max over ranks; value counts all ranks' tokens.
+Under torchrun only the headline workload runs (unless --also-multi).
 """
 from __future__ import annotations
 
@@ -109,6 +114,13 @@ def gate_up_bytes(L, touched) -> int:
     return int(wb + L.T * L.d * 2 + L.T * (L.k + L.S) * L.I * 2)
 
 
+def down_bytes(L, touched) -> int:
+    """Algorithmic HBM bytes of one down GEMM launch: W2 codes and scales of every
+    touched (and shared) expert, H read once and Y written once."""
+    wb = sum(L.experts[e].w2.nbytes + L.experts[e].s2.nbytes for e in list(touched) + list(range(L.E, L.E + L.S)))
+    return int(wb + L.T * (L.k + L.S) * L.I * 2 + L.T * (L.k + L.S) * L.d * 2)
+
+
 def layer_bytes(L, touched) -> int:
     """Algorithmic HBM bytes of one forward: touched experts' weights and scales,
     router weights, x read once and out written once."""
@@ -196,15 +208,18 @@ class ClockSampler:
 # our arm
 # ---------------------------------------------------------------------------
 def time_steps(fn, steps, warmup, flush, stream):
-    """Per-step CUDA-event times (ms) on `stream`, L2 flushed between steps."""
+    """Per-step CUDA-event times (ms) on `stream`; L2 flushed between steps
+    when `flush` is a buffer (None: warm L2, steps back to back)."""
     import torch
     for _ in range(warmup):
-        flush.zero_()
+        if flush is not None:
+            flush.zero_()
         fn()
     torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     for a, b in evs:
-        flush.zero_()
+        if flush is not None:
+            flush.zero_()
         a.record(stream)
         fn()
         b.record(stream)
@@ -212,57 +227,84 @@ def time_steps(fn, steps, warmup, flush, stream):
     return [a.elapsed_time(b) for a, b in evs]
 
 
-def run_ours(args):
+def route_counts(qmoe, dl, x, T, stream):
+    """Per-expert routed-row counts of this batch, from the library's router."""
     import torch
-    import oracle.qmoe_oracle as O  # cpu_baseline leg only
-    from quantized_top_routed_b200 import qmoe, synth
-
-    world, rank = init_dist("nccl")
-    _, _, local = dist_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    peaks = measured_peaks()
-
-    L = synth.make_layer(args.config, T=args.T, seed=args.seed + rank)
-    dl = qmoe.DeviceLayer(L, max_tokens=L.T, device=str(dev))
-    T = L.T
-    stream = torch.cuda.current_stream()
-    out = torch.empty((T, L.d), dtype=torch.int16, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
-
-    # routing of this batch: which experts are touched (bytes never count untouched ones)
+    L = dl.layer
+    dev = dl.x.device
     counts = torch.empty(L.E, dtype=torch.int32, device=dev)
     scratch = [torch.empty((T, L.k), dtype=torch.int32, device=dev),
                torch.empty((T, L.k), dtype=torch.float32, device=dev), counts,
                torch.empty(L.E + 1, dtype=torch.int32, device=dev),
                torch.empty(T * L.k, dtype=torch.int32, device=dev),
                torch.empty((T, L.k), dtype=torch.int32, device=dev)]
-    qmoe.qmoe_route(dl.handle, dl.x, None, T, *scratch, stream)
+    qmoe.qmoe_route(dl.handle, x, None, T, *scratch, stream)
     torch.cuda.synchronize()
-    cnt = counts.cpu().numpy()
-    touched = [int(e) for e in np.nonzero(cnt)[0]]
+    return counts.cpu().numpy().astype(np.int64)
+
+
+def load_report(L, counts):
+    """Realised per-expert load of the batch: the routed-row histogram, and for
+    a Zipf-biased router the exponent s of a least-squares fit
+    log(count) = a - s * log(rank) over the experts that received rows."""
+    from quantized_top_routed_b200 import synth
+    rep = {"counts": [int(c) for c in counts], "touched_experts": int((counts > 0).sum()),
+           "max_over_mean": round(float(counts.max() / max(counts.mean(), 1e-9)), 3)}
+    target = synth.CONFIGS.get(L.name, {}).get("zipf")
+    if target:
+        c = np.sort(counts[counts > 0])[::-1].astype(np.float64)
+        r = np.arange(1, len(c) + 1, dtype=np.float64)
+        slope = np.polyfit(np.log(r), np.log(c), 1)[0] if len(c) > 1 else float("nan")
+        rep.update({"zipf_s_target": target, "zipf_s_fit": round(float(-slope), 3),
+                    "fit": "least squares of log(count) on log(rank), experts with rows"})
+    return rep
+
+
+def compute_dtype_note(L) -> str:
+    if compute_dtype(L) == "f16":
+        return ("f16: every expert is FP8 e4m3, so the grouped GEMMs take fp16 inputs (codes, x rows and H "
+                "convert exactly or with >= bf16 precision); x and H must stay inside |v| < 65504; fp32 accumulation")
+    return "bf16 MMA inputs (dequantised weights, x rows, H), fp32 accumulation"
+
+
+def measure_layer(args, name, T, rank, world, dev, peaks, flush, headline):
+    """Time one workload through qmoe_forward (device buffers, L2 flushed and
+    warm), per-kernel events, the host-buffer entry point, and the roofline of
+    the dominant kernel.  Returns the record (without the CPU baseline)."""
+    import torch
+    from quantized_top_routed_b200 import qmoe, synth
+
+    L = synth.make_layer(name, T=T, seed=args.seed + rank)
+    dl = qmoe.DeviceLayer(L, max_tokens=L.T, device=str(dev))
+    T = L.T
+    stream = torch.cuda.current_stream()
+    out = torch.empty((T, L.d), dtype=torch.int16, device=dev)
+    counts = route_counts(qmoe, dl, dl.x, T, stream)
+    touched = [int(e) for e in np.nonzero(counts)[0]]   # bytes never count untouched experts
+    steps = args.steps if headline else min(args.steps, args.other_steps)
 
     def step():
         qmoe.qmoe_forward(dl.handle, dl.x, T, out, stream)
 
     # ---- timed region ------------------------------------------------------
-    # No per-kernel events here: an event between two launches would undo the
-    # programmatic dependent launches that overlap each kernel's start with
-    # the previous one's tail.
+    # No per-kernel events here, only the step's own pair.
     barrier(dev)
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        times = time_steps(step, args.steps, args.warmup, flush, stream)
+    with ClockSampler(dev.index) as clk:
+        times = time_steps(step, steps, args.warmup, flush, stream)
     torch.cuda.synchronize()
     barrier(dev)
     qmoe.qmoe_check_error(dl.handle, stream)
     ms, value = job_rate(world, T, sum(times) / len(times), dev)
 
+    # warm L2: the same steps back to back without the flush
+    warm = time_steps(step, steps, args.warmup, None, stream)
+    warm_ms, warm_value = job_rate(world, T, sum(warm) / len(warm), dev)
+
     # ---- per-kernel times: the same steps again with an event pair around
     # every launch (L2 flushed between steps as above) ---------------------------
-    prof_steps = min(args.steps, 100)
     qmoe.qmoe_profile(dl.handle, True)
-    time_steps(step, prof_steps, 0, flush, stream)
+    time_steps(step, min(steps, 100), 0, flush, stream)
     stage_ms, calls = qmoe.qmoe_profile_read(dl.handle)
     qmoe.qmoe_profile(dl.handle, False)
 
@@ -274,14 +316,14 @@ def run_ours(args):
         qmoe.qmoe_forward_host(dl.handle, x_host, T, out_host, stream)
 
     barrier(dev)
-    e2e_times = time_steps(e2e_step, args.steps, args.warmup, flush, stream)
+    e2e_times = time_steps(e2e_step, steps, args.warmup, flush, stream)
     barrier(dev)
+    qmoe.qmoe_check_error(dl.handle, stream)
     e2e_ms, e2e_value = job_rate(world, T, sum(e2e_times) / len(e2e_times), dev)
 
     # ---- roofline of the dominant kernel -----------------------------------
     gu_ms = stage_ms["gate_up"] / max(calls, 1)
-    hbm_bound = L.name in ("decode", "tiny")
-    if hbm_bound:
+    if L.name in ("decode", "tiny"):
         algo = gate_up_bytes(L, touched)
         achieved = algo / (gu_ms / 1e3) / 1e9
         roof = {"kernel": "grouped_gemm gate/up (SwiGLU)", "bound": "hbm", "achieved": round(achieved, 1),
@@ -294,30 +336,67 @@ def run_ours(args):
         peak = peaks["bf16_tflops"]
         roof = {"kernel": "grouped_gemm gate/up (SwiGLU)", "bound": "tensor", "achieved": round(achieved, 1),
                 "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "frac_of_sustained_peak": round(achieved / peaks["bf16_tflops_sustained"], 4),
                 "traffic": traffic_from_profiles(L, "gate_up"), "peak_source": peaks["source"],
                 "algorithmic_flops": fl, "avg_launch_ms": round(gu_ms, 5), "timing": ROOF_TIMING}
 
-    result = {
-        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": compute_dtype(L), "data": "synthetic (seeded, shapes of the workload)",
-        "config": {"workload": workload_desc(L), "T": T, "global_batch": world * T, "parallelism": f"replicas x{world}",
-                   "l2": "flushed between timed steps (256 MB write)", "touched_experts": len(touched)},
+    rec = {
+        "value": round(value, 1), "unit": UNIT, "ms_per_step": round(ms, 5), "steps": steps,
+        "dtype": compute_dtype(L), "dtype_note": compute_dtype_note(L),
+        "config": {"workload": workload_desc(L), "T": T, "global_batch": world * T,
+                   "parallelism": f"replicas x{world}", "l2": "flushed between timed steps (256 MB write)",
+                   "touched_experts": len(touched)},
+        "warm_l2": {"value": round(warm_value, 1), "ms_per_step": round(warm_ms, 5),
+                    "note": "the same steps back to back, L2 not flushed"},
         "layer": {"bytes": layer_bytes(L, touched), "flops": layer_flops(L),
                   "hbm_frac": round(layer_bytes(L, touched) / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
                   "tensor_frac": round(layer_flops(L) / (ms / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
                   "stage_ms": {k_: round(v / max(calls, 1), 5) for k_, v in stage_ms.items()}},
         "roofline": roof,
-        "e2e": {"value": round(e2e_value, 1), "unit": UNIT,
+        "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "ms_per_step": round(e2e_ms, 5),
                 "h2d_bytes_per_step": int(T * L.d * 2), "d2h_bytes_per_step": int(T * L.d * 2)},
-        "gpu_launches": qmoe.qmoe_launches_per_forward(dl.handle, T) * args.steps,
+        "gpu_launches": qmoe.qmoe_launches_per_forward(dl.handle, T) * steps,
+        "load": load_report(L, counts),
         "clocks": clk.summary(),
     }
-    if args.sweep and L.name == "decode" and rank == 0:
-        result["sweep"] = sweep_decode(L, dl, flush, stream, peaks)
-    if rank == 0 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(L, O, args)
+    if headline and args.sweep and L.name == "decode" and rank == 0:
+        rec["sweep"] = sweep_decode(L, dl, flush, stream, peaks)
     dl.close()
+    return L, rec
+
+
+def run_ours(args):
+    import torch
+    import oracle.qmoe_oracle as O  # cpu_baseline leg only
+
+    world, rank = init_dist("nccl")
+    _, _, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks = measured_peaks()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    # The headline workload, then (one GPU, default run) the other workloads,
+    # each measured in the same process with its own roofline and baseline.
+    names = [args.config] + [n for n in args.also if n != args.config]
+    if world > 1 and not args.also_multi:
+        names = names[:1]
+    result = None
+    for i, name in enumerate(names):
+        L, rec = measure_layer(args, name, args.T if i == 0 else None, rank, world, dev, peaks, flush, i == 0)
+        if rank == 0 and not args.no_cpu_baseline:
+            rec["cpu_baseline"] = cpu_baseline(L, O, args)
+        del L
+        if i == 0:
+            result = {"metric": METRIC, "value": rec.pop("value"), "unit": UNIT, "n_gpus": world,
+                      "steps": rec.pop("steps"), "warmup": args.warmup, "ms_per_step": rec.pop("ms_per_step"),
+                      "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                      "dtype": rec.pop("dtype"), "data": "synthetic (seeded, shapes of the workload)"}
+            result.update(rec)
+            if len(names) > 1:
+                result["configs"] = {}
+        else:
+            result["configs"][name] = rec
     if rank == 0:
         print(json.dumps(result), flush=True)
     import torch.distributed as dist
@@ -336,15 +415,8 @@ def sweep_decode(L, dl, flush, stream, peaks):
         sub = dataclasses.replace(L, T=T, x=L.x[:T])
         out = torch.empty((T, L.d), dtype=torch.int16, device=dl.x.device)
         xs = dl.x[:T]
-        counts = torch.empty(L.E, dtype=torch.int32, device=dl.x.device)
-        scratch = [torch.empty((T, L.k), dtype=torch.int32, device=dl.x.device),
-                   torch.empty((T, L.k), dtype=torch.float32, device=dl.x.device), counts,
-                   torch.empty(L.E + 1, dtype=torch.int32, device=dl.x.device),
-                   torch.empty(T * L.k, dtype=torch.int32, device=dl.x.device),
-                   torch.empty((T, L.k), dtype=torch.int32, device=dl.x.device)]
-        qmoe.qmoe_route(dl.handle, xs, None, T, *scratch, stream)
-        torch.cuda.synchronize()
-        touched = [int(e) for e in np.nonzero(counts.cpu().numpy())[0]]
+        counts = route_counts(qmoe, dl, xs, T, stream)
+        touched = [int(e) for e in np.nonzero(counts)[0]]
         fwd = lambda: qmoe.qmoe_forward(dl.handle, xs, T, out, stream)  # noqa: E731
         times = time_steps(fwd, 200, 5, flush, stream)
         qmoe.qmoe_profile(dl.handle, True)
@@ -354,9 +426,11 @@ def sweep_decode(L, dl, flush, stream, peaks):
         ms = sum(times) / len(times)
         lb = layer_bytes(sub, touched)
         gu = stage_ms["gate_up"] / max(calls, 1)
+        dn = stage_ms["down"] / max(calls, 1)
         rows.append({"T": T, "tokens_per_s": round(T / (ms / 1e3), 1), "ms": round(ms, 5),
                      "touched_experts": len(touched), "layer_hbm_frac": round(lb / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
                      "gate_up_hbm_frac": round(gate_up_bytes(sub, touched) / (gu / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+                     "down_hbm_frac": round(down_bytes(sub, touched) / (dn / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
                      "stage_ms": {k_: round(v / max(calls, 1), 5) for k_, v in stage_ms.items()}})
     return rows
 
@@ -389,16 +463,30 @@ def oracle_sample_tokens(L, n, step):
     return np.array([(step * n + i) % L.T for i in range(n)])
 
 
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
 def cpu_baseline(L, O, args):
+    """The fp64 oracle as it stands, single-threaded, on a bounded sample of the
+    same batch: whole tokens (routing, dequantisation of their experts, the
+    expert FFNs and the combine), one oracle call per token, until about
+    --cpu-seconds have passed (at least one token)."""
     from threadpoolctl import threadpool_limits
-    n = args.cpu_tokens
+    n, dt = 0, 0.0
     with threadpool_limits(limits=1):
         t0 = time.perf_counter()
-        O.forward(L, tokens=oracle_sample_tokens(L, n, 0))
-        dt = time.perf_counter() - t0
-    return {"value": round(n / dt, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{n} tokens of the same batch (routing, dequantisation of the touched experts "
-                      f"and the expert FFNs in float64, single thread), {dt:.1f} s"}
+        while n < args.cpu_tokens and (n == 0 or dt < args.cpu_seconds):
+            O.forward(L, tokens=oracle_sample_tokens(L, 1, n))
+            n += 1
+            dt = time.perf_counter() - t0
+    return {"value": round(n / dt, 4), "unit": UNIT, "cores": 1, "host_cores": host_cores(),
+            "omp_num_threads": os.environ.get("OMP_NUM_THREADS"), "kind": "oracle",
+            "sample": f"{n} tokens of the same batch, one oracle call each (routing, dequantisation of the "
+                      f"token's experts, the expert FFNs and the combine in float64), one thread, {dt:.1f} s"}
 
 
 def oracle_task(O, L, step):
@@ -454,12 +542,19 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--config", default="decode", choices=("tiny", "decode", "prefill", "fine", "mixed"))
+    ap.add_argument("--config", default="decode", choices=("tiny", "decode", "prefill", "fine", "mixed"),
+                    help="the headline workload (default: decode, T=256)")
+    ap.add_argument("--also", nargs="*", default=["prefill", "fine", "mixed"],
+                    choices=("tiny", "decode", "prefill", "fine", "mixed"),
+                    help="further workloads measured in the same run (one GPU) under 'configs'")
+    ap.add_argument("--also-multi", action="store_true", help="measure --also workloads under torchrun too")
+    ap.add_argument("--other-steps", type=int, default=30, help="timed steps of each --also workload (at most --steps)")
     ap.add_argument("--T", type=int, default=None, help="tokens per step (default: the workload's)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-sweep", dest="sweep", action="store_false")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-tokens", type=int, default=48, help="tokens in the timed oracle sample")
+    ap.add_argument("--cpu-tokens", type=int, default=48, help="at most this many tokens in the timed oracle sample")
+    ap.add_argument("--cpu-seconds", type=float, default=8.0, help="time budget of the oracle sample per workload")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

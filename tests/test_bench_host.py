@@ -58,3 +58,25 @@ def test_traffic_is_dropped_when_the_kernel_source_changes(tmp_path, monkeypatch
     assert bench.traffic_from_profiles(L, "down") is None
     (csrc / "gemm.cu").write_text("kernel v2")
     assert bench.traffic_from_profiles(L, "gate_up") is None
+
+
+def test_down_bytes_of_the_fine_shape_by_hand():
+    L = synth.make_layer("fine", T=8, d=256, E=4, k=2, I=128, S=1)
+    touched = [1, 3]
+    # INT4 g128 W2: codes d x I / 2 bytes, bf16 scales d x I/128 x 2 bytes; touched + shared experts
+    w = 3 * (256 * 128 // 2 + 256 * (128 // 128) * 2)
+    h = 8 * (2 + 1) * 128 * 2
+    y = 8 * (2 + 1) * 256 * 2
+    assert bench.down_bytes(L, touched) == w + h + y
+
+
+def test_load_report_recovers_a_zipf_exponent():
+    import numpy as np
+    L = types.SimpleNamespace(name="fine")               # a Zipf(1.2)-biased workload
+    counts = np.round(1e5 * np.arange(1, 65, dtype=np.float64) ** -1.2).astype(np.int64)
+    rep = bench.load_report(L, np.random.default_rng(0).permutation(counts))
+    assert rep["zipf_s_target"] == 1.2
+    assert abs(rep["zipf_s_fit"] - 1.2) < 0.01
+    assert rep["touched_experts"] == 64 and sum(rep["counts"]) == counts.sum()
+    flat = bench.load_report(types.SimpleNamespace(name="decode"), np.full(8, 5))
+    assert "zipf_s_fit" not in flat and flat["max_over_mean"] == 1.0

@@ -93,10 +93,15 @@ def check_route_from_x(dl, T):
 
 
 def check_forward(dl, T, tokens=None):
-    """Layer output against the oracle on the GPU's routing; returns (rel_l2, max_abs, unsafe)."""
+    """Layer output against the oracle on the GPU's routing; returns (rel_l2, max_abs, unsafe).
+
+    tokens: None (every token), an index array, or a callable that picks the
+    tokens from the GPU's routing result."""
     L = sub_layer(dl.layer, T)
     g, unsafe = check_route_from_x(dl, T)
     out = run_forward(dl, T)
+    if callable(tokens):
+        tokens = tokens(g, L)
     tok = np.arange(T) if tokens is None else np.asarray(tokens)
     ref = O.forward(L, tokens=tok, idx_override=g["idx"][tok])
     got = out[tok]
@@ -112,6 +117,29 @@ def sample_tokens(T, n=48, seed=0):
     rng = np.random.default_rng(seed)
     pick = set(rng.choice(T, size=min(n, T), replace=False).tolist()) | {0, T - 1}
     return np.array(sorted(pick))
+
+
+def covering_tokens(block=64, n_random=16):
+    """Token picker for full-size layers: for every expert segment of the
+    schedule (routed experts from the GPU's offsets, then the identity
+    segments of the shared experts), the token of the first row of every
+    `block`-row block and of the segment's last row, so every token block of
+    the grouped GEMMs (token blocks are at most 128 rows and a multiple of 16)
+    contributes a checked output, ragged last blocks included; plus a few
+    random tokens."""
+    def pick(g, L):
+        tok = set(sample_tokens(L.T, n_random).tolist())
+        st, off = g["sorted_token"], g["offsets"]
+        for e in range(L.E):
+            lo, hi = int(off[e]), int(off[e + 1])
+            if hi > lo:
+                tok.update(int(st[p]) for p in range(lo, hi, block))
+                tok.add(int(st[hi - 1]))
+        if L.S:
+            tok.update(range(0, L.T, block))
+            tok.add(L.T - 1)
+        return np.array(sorted(tok))
+    return pick
 
 
 # ---------------------------------------------------------------------------
@@ -168,21 +196,21 @@ def test_decode_sweep(decode_layer, T):
 def test_prefill_full_size_sampled():
     L = synth.make_layer("prefill")
     dl = qmoe.DeviceLayer(L)
-    check_forward(dl, L.T, tokens=sample_tokens(L.T, 40))
+    check_forward(dl, L.T, tokens=covering_tokens(64))
     dl.close()
 
 
 def test_fine_shared_zipf_full_size_sampled():
     L = synth.make_layer("fine")
     dl = qmoe.DeviceLayer(L)
-    check_forward(dl, L.T, tokens=sample_tokens(L.T, 64))
+    check_forward(dl, L.T, tokens=covering_tokens(64))
     dl.close()
 
 
 def test_mixed_precision_full_size_sampled():
     L = synth.make_layer("mixed")
     dl = qmoe.DeviceLayer(L)
-    check_forward(dl, L.T, tokens=sample_tokens(L.T, 48))
+    check_forward(dl, L.T, tokens=covering_tokens(128))
     dl.close()
 
 
@@ -226,6 +254,7 @@ def test_k_equals_E_uniform_router_is_mean_of_experts():
     x = O.bf16_to_f64(L.x)
     mean = np.mean([O.expert_ffn(x, *O.dequantize_expert(ex, L.d, L.I), L.I) for ex in L.experts], axis=0)
     assert O.rel_l2(out, mean) <= REL_L2
+    assert float(np.abs(out - mean).max()) <= MAX_ABS
     dl.close()
 
 

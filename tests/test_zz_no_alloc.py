@@ -3,8 +3,8 @@ no handle, no allocation) against qmoe_route on the same inputs.
 
 Both run the same router kernel with the same d-split, so expert indices
 and gates must agree bit for bit.  Two consecutive calls with different
-activations check that nothing from the first call (partial logits, the
-per-tile counters) leaks into the second.  The file is collected last so it
+activations check that nothing from the first call (the partial logits
+left in the shared scratch array) leaks into the second.  The file is collected last so it
 also runs after every other GPU test has used the library in this process.
 """
 import numpy as np
