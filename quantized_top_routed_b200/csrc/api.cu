@@ -103,6 +103,7 @@ struct qmoe_handle {
   uint16_t *Xp = nullptr, *H = nullptr, *Y = nullptr, *x_stage = nullptr, *out_stage = nullptr;
   int* err = nullptr;
   int zpart_split_max = 1;
+  long long wait_limit = kWaitLimit;     // bound of the grouped GEMMs' mbarrier waits (SM cycles)
   // profiling
   bool profiling = false;
   int profiled_calls = 0;
@@ -394,6 +395,7 @@ qmoe_status qmoe_forward(qmoe_handle* h, const uint16_t* x, int32_t T, uint16_t*
   g.seg_cnt = h->seg_cnt;
   g.n_seg = c.E + c.n_shared;
   g.err = h->err;
+  g.wait_limit = h->wait_limit;
   for (int mat = 0; mat < 2; ++mat) {
     StageTimer tm(h, s, mat == 0 ? QMOE_STAGE_GATE_UP : QMOE_STAGE_DOWN);
     g.mat = mat;

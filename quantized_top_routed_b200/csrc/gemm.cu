@@ -15,92 +15,91 @@
 //   B (N x K) = BN consecutive rows of the expert's segment in the permuted
 //               activations (x rows in schedule order, or H), loaded by TMA
 //               tiles (two per K stage) into 128-byte-swizzled shared memory;
-//   D (M x N) = fp32 accumulators in tensor memory, double buffered.
+//   D (M x N) = fp32 accumulators in tensor memory.
 // Weights are the M side because an expert usually has few tokens: the
 // weight stream is what the kernel moves.  Raw code tiles arrive by TMA bulk
-// copy into a ring sized per weight format (no instruction cost per byte);
-// the dequantisation warps read them with conflict-free 16-byte shared
-// loads.  Every role signals once per warp per stage, so the SM's issue
-// slots go to the dequantisation arithmetic.  INT4 group scales are applied
-// during dequantisation (bf16(q*s), one rounding); INT8 and FP8 per-channel
-// scales are applied to the fp32 accumulator in the epilogue (exact
-// factoring).
+// copy into a ring sized per weight format; the dequantisation warps read
+// them with conflict-free 16-byte shared loads.  INT4 group scales are
+// applied during dequantisation (bf16(q*s), one rounding); INT8 and FP8
+// per-channel scales are applied to the fp32 accumulator in the epilogue
+// (exact factoring).
+//
+// Issue rate.  One warp issues a tcgen05.mma about every 60-100 cycles
+// whatever N is, while an M=128, N<=64, K=16 MMA needs far less tensor time;
+// the rate grows with the number of warps issuing.  So the K stages of a
+// tile are split into two classes (even and odd stage index), each with its
+// own issuer warp accumulating into its own partial accumulator in TMEM; the
+// epilogue adds the two partials in a fixed order (deterministic).
 //
 // Persistent CTAs (one per SM) walk the tile list (segment, 128-row weight
 // block, BN-row token block) built on the device by the schedule kernel;
-// one launch handles the experts of one weight format.  A CTA works on G
-// tiles at a time (G = 2 for token blocks of up to 32 rows): K stage k of
-// all G tiles forms one super-stage, produced, signalled and released as a
-// unit, and each tile has its own MMA warp and accumulator, so one warp's
-// barrier wait and commit overlap the other warp's MMAs -- a single issuing
-// thread leaves the tensor pipe idle for several hundred cycles per stage,
-// and every barrier operation costs a dequantisation warp ~200 cycles.
+// one launch handles the experts of one weight format.  Everything a class
+// touches is private to it: dequantisation group c, issuer c, partial c, and
+// half of the raw ring and of the stage ring (A in TMEM, B in shared memory).
+// So every ring slot has one producer and one consumer that both walk its
+// uses in order, and a parity wait can never be two phases behind.
 // Warp roles, all synchronised through mbarriers:
 //   warp 0       : TMEM allocation; lane 0 streams raw weight tiles (bulk copy)
 //   warp 1       : lane 0 issues the B tile loads (TMA)
-//   warps 2, 3   : lane 0 of warp 2 + j issues the MMAs and commits of tile j
-//   warps 4..11  : dequantise A into TMEM, as 2 groups of 4 warps that take
-//                  alternate super-stages (so two are in flight); warp w
-//                  owns TMEM lane quarter w % 4, one weight row per thread
-//   warps 12..15 : epilogue (TMEM -> registers -> scales / SwiGLU -> bf16)
-// Every wait is bounded: a role that waits ~1 s raises an abort flag, all
-// roles drain what they issued, TMEM is freed and the error word is set.
+//   warps 2, 3   : MMA issuers of classes 0 and 1 (warp-uniform loops, lane 0 issues)
+//   warps 4..11  : dequantise A into TMEM, group c = warps 4 + 4c .. 7 + 4c;
+//                  warp w owns TMEM lane quarter w % 4, one weight row per thread
+//   warps 12..15 : epilogue (TMEM -> registers -> sum of partials, scales,
+//                  SwiGLU -> bf16)
+// Every wait is bounded (GemmArgs::wait_limit cycles): a role that waits too
+// long raises an abort flag, all roles drain what they issued (the producers
+// on barriers that only their own copies complete, the issuers on a commit),
+// TMEM is freed and the error word is set.
 #include <cuda.h>
 #include <cuda_fp16.h>
-
-#include <type_traits>
 
 #include "qmoe_internal.cuh"
 
 namespace qmoe {
 namespace {
 
-constexpr int kNDQ = 8;                        // dequantisation warps
-constexpr int kGroups = kNDQ / 4;              // groups of 4 warps; group g converts super-stages g, g+2, ...
-constexpr int kKW = kBK;                       // K elements one dequant thread converts per stage (its row)
-constexpr int kHalf = kKW / 2;                 // converted and stored in two halves
 constexpr int kRawWarp = 0, kBWarp = 1, kMmaWarp0 = 2;
-constexpr int kMaxG = 2;                       // tiles in flight per CTA (one MMA warp each)
-constexpr int kDQWarp0 = kMmaWarp0 + kMaxG;
-constexpr int kEpiWarp0 = kDQWarp0 + kNDQ;
+constexpr int kCls = 2;                        // stage classes (issuer warp + dequantisation group each)
+constexpr int kDQWarp0 = kMmaWarp0 + kCls;     // first dequantisation warp
+constexpr int kEpiWarp0 = kDQWarp0 + 4 * kCls;
 constexpr int kThreads = 32 * (kEpiWarp0 + 4);
+constexpr int kKW = kBK;                       // K elements one dequant thread converts per item (its row)
 constexpr int kTabMax = kMaxE + kMaxShared + 1;
 constexpr uint32_t kTmemCols = 512;
 // Poll back-off (ns) of the roles that wait off the critical path: the
-// producers run ahead of the ring and the epilogue waits a whole tile.
+// producers run ahead of the rings and the epilogue waits a whole tile.
 constexpr uint32_t kSleepRaw = 128, kSleepB = 64, kSleepEpi = 256;
 
 template <int FMT>
 struct FmtCfg {
   static constexpr int SB = FMT == QMOE_W_INT4_G128 ? 128 * 64 + 256 : 128 * 128;  // bytes of a raw tile
-  static constexpr int NC = FMT == QMOE_W_INT4_G128 ? kHalf / 32 : kHalf / 16;      // 16-byte chunks per half row
+  static constexpr int QC = FMT == QMOE_W_INT4_G128 ? 1 : 2;    // 16-byte chunks per quarter row (16 pairs)
 };
 
 template <int BN, int FMT>
 struct Cfg {
-  static constexpr int G = BN <= 32 ? 2 : 1;                      // tiles in flight
-  static constexpr int A_COL0 = 2 * G * BN;                       // TMEM: 2 accumulators per tile, then A
-  static constexpr int SA0 = ((int)kTmemCols - A_COL0) / 64;
-  static constexpr int SP = (SA0 > 7 ? 7 : SA0) / G;              // super-stage slots (G stages each)
-  static constexpr int SA = SP * G;                               // A/B stage slots (TMEM + smem)
-  static constexpr int B_STAGE = BN * 256;                        // BN rows x 128 K bf16
-  static constexpr int STAGING = BN * 256;                        // epilogue staging
-  static constexpr int SLOT = (FmtCfg<FMT>::SB + 127) & ~127;     // raw ring slot
+  static constexpr int NBUF = BN <= 32 ? 2 : 1;                      // accumulator sets (double buffer)
+  static constexpr int ACC = NBUF * kCls * BN;                       // TMEM columns of the accumulators
+  static constexpr int SH0 = ((int)kTmemCols - ACC) / 64 / kCls;
+  static constexpr int SH = SH0 > 3 ? 3 : SH0;                       // stage slots per class
+  static constexpr int SA = kCls * SH;                               // stage ring: A (TMEM) + B (smem)
+  static constexpr int B_STAGE = BN * 256;                           // BN rows x 128 K bf16
+  static constexpr int STAGING = 4 * 16 * (BN <= 32 ? BN / 16 : 1) * 64;   // epilogue staging (4 warps)
+  static constexpr int SLOT = (FmtCfg<FMT>::SB + 127) & ~127;        // raw ring slot
   static constexpr int FIXED = SA * B_STAGE + STAGING + 6 * 1024;
-  static constexpr int R0 = (224 * 1024 - FIXED) / SLOT;
-  static constexpr int RP = (R0 > 16 ? 16 : R0) / G;              // raw ring: super-stage slots
-  static constexpr int R = RP * G;                                // raw ring: tile slots
+  static constexpr int R0 = (224 * 1024 - FIXED) / SLOT / kCls;
+  static constexpr int RH = R0 > 8 ? 8 : R0;                         // raw slots per class
+  static constexpr int R = kCls * RH;
   static constexpr int OFF_B = 0;
   static constexpr int OFF_RAW = OFF_B + SA * B_STAGE;
   static constexpr int OFF_STG = OFF_RAW + R * SLOT;
   static constexpr int OFF_TAB = OFF_STG + STAGING;
   static constexpr int OFF_BAR = (OFF_TAB + 3 * kTabMax * 4 + 127) & ~127;
-  static constexpr int NUM_BARS = 2 * SP + 2 * RP + 4 * G + G;
+  static constexpr int NUM_BARS = 3 * SA + 2 * R + 2 * NBUF + kCls;
   static constexpr int OFF_MISC = (OFF_BAR + NUM_BARS * 8 + 15) & ~15;
-  static constexpr int SMEM = OFF_MISC + 16 + 1024;               // + alignment slack
-  static_assert(RP >= 3 && SP >= 3, "rings too shallow");
-  static_assert(G <= kMaxG, "MMA warps");
-  static_assert(A_COL0 + SA * 64 <= (int)kTmemCols, "TMEM budget");
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;                  // + alignment slack
+  static_assert(RH >= 2 && SH >= 2, "rings too shallow");
+  static_assert(ACC + SA * 64 <= (int)kTmemCols, "TMEM budget");
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(B_STAGE % 1024 == 0 && OFF_RAW % 1024 == 0 && OFF_BAR % 8 == 0 && OFF_MISC % 16 == 0,
                 "alignment");
@@ -179,11 +178,11 @@ __device__ __forceinline__ void deq_fp8_f16_word(uint32_t w, uint32_t* o) {
       : "r"(w));
 }
 
-// This thread's 16-byte chunks (K order) -> kHalf / 2 bf16 (or fp16) pairs.
-template <int FMT>
-__device__ __forceinline__ void dequant_slice(const uint4 (&w)[FmtCfg<FMT>::NC], uint32_t sbits, uint32_t* av) {
+// NCHK of this thread's 16-byte chunks (K order) -> bf16 (or fp16) pairs.
+template <int FMT, int NCHK>
+__device__ __forceinline__ void dequant_chunks(const uint4* w, uint32_t sbits, uint32_t* av) {
 #pragma unroll
-  for (int c = 0; c < FmtCfg<FMT>::NC; ++c) {
+  for (int c = 0; c < NCHK; ++c) {
     if constexpr (FMT == QMOE_W_INT4_G128) {
       const uint32_t s2 = sbits | (sbits << 16);
       deq_int4_word(w[c].x, s2, &av[16 * c + 0]);
@@ -209,7 +208,9 @@ __device__ __forceinline__ void dequant_slice(const uint4 (&w)[FmtCfg<FMT>::NC],
   }
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+// silu(g) * u with the fast exponential and division: the layer's output
+// tolerance is far above their few-ulp error.
+__device__ __forceinline__ float swiglu_f(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
 __device__ __forceinline__ uint16_t f2bf(float f) {
   const __nv_bfloat16 b = __float2bfloat16_rn(f);
@@ -231,12 +232,13 @@ __device__ __forceinline__ void tma_tile2d(uint32_t dst, const CUtensorMap* map,
 }
 
 // Warp-uniform bounded wait: every lane polls, the warp proceeds together.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, long long lim) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, lim));
 }
 // The same for roles off the critical path: back off between polls.
-__device__ __forceinline__ bool warp_wait_backoff(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t ns) {
-  return __all_sync(0xffffffffu, mbar_wait_backoff(bar, parity, abort, ns));
+__device__ __forceinline__ bool warp_wait_backoff(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t ns,
+                                                  long long lim) {
+  return __all_sync(0xffffffffu, mbar_wait_backoff(bar, parity, abort, ns, lim));
 }
 
 template <int BN, int MAT, int FMT>
@@ -244,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap act_map) {
   using C = Cfg<BN, FMT>;
   using F = FmtCfg<FMT>;
-  constexpr int G = C::G;
+  constexpr int SH = C::SH, RH = C::RH, NBUF = C::NBUF;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sB = smem + C::OFF_B;
@@ -254,34 +256,41 @@ __global__ void __launch_bounds__(kThreads, 1)
   int32_t* s_seg_off = tab_off + kTabMax;
   int32_t* s_seg_cnt = s_seg_off + kTabMax;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* full = bars;                      // [SP] B landed + A in TMEM, per super-stage
-  uint64_t* empty = full + C::SP;             // [SP] MMAs done with the super-stage
-  uint64_t* raw_full = empty + C::SP;         // [RP] raw tiles of a super-stage landed
-  uint64_t* raw_empty = raw_full + C::RP;     // [RP] raw tiles consumed
-  uint64_t* acc_full = raw_empty + C::RP;     // [G][2] accumulator of tile lane j, buffer b
-  uint64_t* acc_empty = acc_full + 2 * G;     // [G][2]
-  uint64_t* drain = acc_empty + 2 * G;        // [G]
+  uint64_t* full = bars;                      // [SA] A of the item in TMEM (one arrival per dequant warp)
+  uint64_t* bfull = full + C::SA;             // [SA] B tiles of the item landed (TMA bytes only)
+  uint64_t* empty = bfull + C::SA;            // [SA] MMAs done with the slot
+  uint64_t* raw_full = empty + C::SA;         // [R] raw tile of the item landed
+  uint64_t* raw_empty = raw_full + C::R;      // [R] raw tile consumed
+  uint64_t* acc_full = raw_empty + C::R;      // [NBUF] both partials of the tile complete
+  uint64_t* acc_empty = acc_full + NBUF;      // [NBUF] the epilogue has read the partials
+  uint64_t* drain = acc_empty + NBUF;         // [kCls] abort path of the issuers
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_seg = a.n_seg;
   const int KS = a.K / kBK;
+  const long long lim = a.wait_limit;
+  // Items of a class: stage ks of the CTA's tile q with ks = c (mod 2) has
+  // class index q * ncls(c) + ks / 2; it uses stage slot c * SH + index % SH
+  // and raw slot c * RH + index % RH.
+  auto ncls = [&](int c) { return (KS + 1 - c) >> 1; };
 
   if (tid == 0) {
-    for (int s = 0; s < C::SP; ++s) {
-      mbar_init(&full[s], 1 + 4);      // B producer expect_tx + one arrival per warp of a dequant group
-      mbar_init(&empty[s], G);         // one commit per tile lane
+    for (int s = 0; s < C::SA; ++s) {
+      mbar_init(&full[s], 4);
+      mbar_init(&bfull[s], 1);
+      mbar_init(&empty[s], 1);
     }
-    for (int r = 0; r < C::RP; ++r) {
+    for (int r = 0; r < C::R; ++r) {
       mbar_init(&raw_full[r], 1);
       mbar_init(&raw_empty[r], 4);
     }
-    for (int b = 0; b < 2 * G; ++b) {
-      mbar_init(&acc_full[b], 1);
+    for (int b = 0; b < NBUF; ++b) {
+      mbar_init(&acc_full[b], kCls);   // one arrival per issuer
       mbar_init(&acc_empty[b], 4);     // one arrival per epilogue warp
     }
-    for (int j = 0; j < G; ++j) mbar_init(&drain[j], 1);
+    for (int c = 0; c < kCls; ++c) mbar_init(&drain[c], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -302,258 +311,257 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total = tab_off[n_seg];
-  // This CTA's tiles: blockIdx.x + i * gridDim.x for i < nt, taken G at a
-  // time.  A group of gq tiles is processed as KS super-stages; super-stage
-  // ks holds K stage ks of every tile of the group (tile j in stage slot j of
-  // the super-stage slot) and is produced, signalled and released as a unit.
+  // This CTA's tiles: blockIdx.x + q * gridDim.x for q < nt.
   const int nt = (int)blockIdx.x < total ? (total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
-  auto tile_of = [&](int i) { return decode_tile((int)blockIdx.x + i * (int)gridDim.x, tab_off, s_seg_off,
+  auto tile_of = [&](int q) { return decode_tile((int)blockIdx.x + q * (int)gridDim.x, tab_off, s_seg_off,
                                                  s_seg_cnt, n_seg, BN); };
 
   if (warp == kRawWarp) {
-    // ---------------- raw weight tiles: one bulk copy per tile per K stage ----------------
-    uint32_t rc = 0, r = 0, ph = 0;         // super-stages issued, ring slot, slot parity
+    // ---------------- raw weight tiles: one bulk copy per item ----------------
     bool ok = true;
-    for (int q0 = 0; q0 < nt && ok; q0 += G) {
-      const int gq = min(G, nt - q0);
-      const uint8_t* src[G];
-#pragma unroll
-      for (int j = 0; j < G; ++j) {
-        if (j < gq) {
-          const Tile t = tile_of(q0 + j);
-          src[j] = a.experts[t.seg].w[MAT] + (size_t)t.mb * KS * F::SB;
-        }
-      }
+    uint32_t issued[kCls] = {0, 0};
+    for (int q = 0; q < nt && ok; ++q) {
+      const Tile t = tile_of(q);
+      const uint8_t* src = a.experts[t.seg].w[MAT] + (size_t)t.mb * KS * F::SB;
       for (int ks = 0; ks < KS; ++ks) {
-        ok = warp_wait_backoff(&raw_empty[r], ph ^ 1, abort_flag, kSleepRaw);
+        const int c = ks & 1;
+        const uint32_t i = (uint32_t)(q * ncls(c) + (ks >> 1));
+        const uint32_t r = c * RH + i % RH, ph = (i / RH) & 1;
+        ok = warp_wait_backoff(&raw_empty[r], ph ^ 1, abort_flag, kSleepRaw, lim);
         if (!ok) break;
         if (lane == 0) {
-          mbar_arrive_expect_tx(&raw_full[r], (uint32_t)(gq * F::SB));
-#pragma unroll
-          for (int j = 0; j < G; ++j)
-            if (j < gq) bulk_g2s(sRaw + (r * G + j) * C::SLOT, src[j] + (size_t)ks * F::SB, F::SB, &raw_full[r]);
+          mbar_arrive_expect_tx(&raw_full[r], (uint32_t)F::SB);
+          bulk_g2s(sRaw + r * C::SLOT, src + (size_t)ks * F::SB, F::SB, &raw_full[r]);
         }
         __syncwarp();
-        ++rc;
-        if (++r == (uint32_t)C::RP) { r = 0; ph ^= 1; }
+        issued[c] = i + 1;
       }
     }
-    // wait for copies that may still be in flight before the CTA can exit
+    // copies that may still be in flight complete before the CTA can exit
     if (lane == 0) {
-      const uint32_t first = rc > (uint32_t)C::RP ? rc - C::RP : 0;
-      for (uint32_t i = first; i < rc; ++i) mbar_wait_drain(&raw_full[i % C::RP], (i / C::RP) & 1);
+      for (int c = 0; c < kCls; ++c) {
+        const uint32_t first = issued[c] > (uint32_t)RH ? issued[c] - RH : 0;
+        for (uint32_t i = first; i < issued[c]; ++i) mbar_wait_drain(&raw_full[c * RH + i % RH], (i / RH) & 1);
+      }
     }
     __syncwarp();
   } else if (warp == kBWarp) {
-    // ---------------- B rows: two TMA tiles per tile per K stage ----------------
-    uint32_t sc = 0, s = 0, ph = 0;
+    // ---------------- B rows: two TMA tiles per item ----------------
     bool ok = true;
-    for (int q0 = 0; q0 < nt && ok; q0 += G) {
-      const int gq = min(G, nt - q0);
-      int row0[G];
-#pragma unroll
-      for (int j = 0; j < G; ++j) row0[j] = j < gq ? tile_of(q0 + j).row0 : 0;
+    uint32_t issued[kCls] = {0, 0};
+    for (int q = 0; q < nt && ok; ++q) {
+      const int row0 = tile_of(q).row0;
       for (int ks = 0; ks < KS; ++ks) {
-        ok = warp_wait_backoff(&empty[s], ph ^ 1, abort_flag, kSleepB);
+        const int c = ks & 1;
+        const uint32_t i = (uint32_t)(q * ncls(c) + (ks >> 1));
+        const uint32_t s = c * SH + i % SH, ph = (i / SH) & 1;
+        ok = warp_wait_backoff(&empty[s], ph ^ 1, abort_flag, kSleepB, lim);
         if (!ok) break;
         if (lane == 0) {
-          mbar_arrive_expect_tx(&full[s], (uint32_t)(gq * C::B_STAGE));
-#pragma unroll
-          for (int j = 0; j < G; ++j) {
-            if (j < gq) {
-              const uint32_t dst = smem_u32(sB + (s * G + j) * C::B_STAGE);
-              tma_tile2d(dst, &act_map, ks * kBK, row0[j], &full[s]);
-              tma_tile2d(dst + BN * 128, &act_map, ks * kBK + 64, row0[j], &full[s]);
-            }
-          }
+          const uint32_t dst = smem_u32(sB + s * C::B_STAGE);
+          mbar_arrive_expect_tx(&bfull[s], (uint32_t)C::B_STAGE);
+          tma_tile2d(dst, &act_map, ks * kBK, row0, &bfull[s]);
+          tma_tile2d(dst + BN * 128, &act_map, ks * kBK + 64, row0, &bfull[s]);
         }
         __syncwarp();
-        ++sc;
-        if (++s == (uint32_t)C::SP) { s = 0; ph ^= 1; }
+        issued[c] = i + 1;
       }
     }
+    // bfull completes on the TMA bytes alone, so this drain ends when the
+    // copies have landed, even after an abort
     if (lane == 0) {
-      const uint32_t first = sc > (uint32_t)C::SP ? sc - C::SP : 0;
-      for (uint32_t i = first; i < sc; ++i) mbar_wait_drain(&full[i % C::SP], (i / C::SP) & 1);
+      for (int c = 0; c < kCls; ++c) {
+        const uint32_t first = issued[c] > (uint32_t)SH ? issued[c] - SH : 0;
+        for (uint32_t i = first; i < issued[c]; ++i) mbar_wait_drain(&bfull[c * SH + i % SH], (i / SH) & 1);
+      }
     }
     __syncwarp();
   } else if (warp < kDQWarp0) {
-    // ---------------- MMA issuer of tile lane j (lane 0 alone) ----------------
-    // A tight single-thread loop: the tensor pipe takes the next MMA only when
-    // the previous one is nearly done, so any work between MMAs is exposed.
-    const int j = warp - kMmaWarp0;
-    if (j < G && lane == 0) {
-      const uint64_t bdesc0 = smem_desc_sw128(smem_u32(sB + j * C::B_STAGE));
-      const uint32_t a_tmem0 = tmem_base + C::A_COL0 + (uint32_t)(j * 64);
-      bool ok = true;
-      for (int q0 = 0, q = 0; q0 < nt && ok; q0 += G, ++q) {
-        const int gq = min(G, nt - q0);
-        if (j >= gq) break;
-        const Tile t = tile_of(q0 + j);
-        const int b = q & 1;
-        ok = mbar_wait(&acc_empty[2 * j + b], ((q >> 1) & 1) ^ 1, abort_flag);
-        if (!ok) break;
+    // ---------------- MMA issuer of class c ----------------
+    // Stages ks = c, c + 2, ... of every tile, accumulated into partial c of
+    // the tile's accumulator set.  The loop runs on the whole warp; lane 0
+    // issues.
+    const int c = warp - kMmaWarp0;
+    const uint64_t bdesc0 = smem_desc_sw128(smem_u32(sB));
+    const uint32_t a_tmem0 = tmem_base + C::ACC;
+    const uint32_t leader = lane == 0;         // the lane that issues every MMA and commit of this warp
+    const int nc = ncls(c);
+    bool ok = true;
+    for (int q = 0; q < nt && ok; ++q) {
+      const Tile t = tile_of(q);
+      const uint32_t idesc = idesc_bf16_m128(max(16, (t.nvalid + 15) & ~15), FMT == kFmtFp8F16);
+      const int b = NBUF == 2 ? (q & 1) : 0;    // accumulator set of this tile
+      const int use = NBUF == 2 ? (q >> 1) : q;  // its use count before this tile
+      // the epilogue has read this set's previous tile
+      if (!(ok = warp_wait(&acc_empty[b], (use & 1) ^ 1, abort_flag, lim))) break;
+      const uint32_t d_tmem = tmem_base + (uint32_t)((b * kCls + c) * BN);
+      for (int ks = c; ks < KS; ks += 2) {
+        const uint32_t i = (uint32_t)(q * nc + (ks >> 1));
+        const uint32_t s = c * SH + i % SH, ph = (i / SH) & 1;
+        if (!(ok = warp_wait(&bfull[s], ph, abort_flag, lim))) break;
+        if (!(ok = warp_wait(&full[s], ph, abort_flag, lim))) break;
         tc_fence_after();
-        const uint32_t idesc = idesc_bf16_m128(max(16, (t.nvalid + 15) & ~15), FMT == kFmtFp8F16);
-        const uint32_t d_tmem = tmem_base + (uint32_t)((2 * j + b) * BN);
-        const int u0 = q * KS;                 // super-stage index of this group's first K stage
-        uint32_t s = (uint32_t)(u0 % C::SP), ph = (uint32_t)((u0 / C::SP) & 1);
-        for (int ks = 0; ks < KS; ++ks) {
-          if (!mbar_wait(&full[s], ph, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          // Descriptors of this stage: only the start-address field moves
-          // (16-byte units), so each MMA's operands are one add away.
-          const uint64_t bdesc = bdesc0 + (uint64_t)(s * (G * C::B_STAGE >> 4));
-          const uint32_t a_tmem = a_tmem0 + s * (G * 64);
+        // Descriptors of this slot: only the start-address field moves
+        // (16-byte units), so each MMA's operands are one add away.
+        const uint64_t bdesc = bdesc0 + (uint64_t)(s * (C::B_STAGE >> 4));
+        const uint32_t a_tmem = a_tmem0 + s * 64;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_bf16_ts(d_tmem, a_tmem + kk * 8, bdesc + (uint64_t)((kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2),
-                        idesc, (ks | kk) != 0);
-          mma_commit(&empty[s]);
-          for (int e = gq; e < G; ++e) mma_commit(&empty[s]);   // stand in for absent tile lanes
-          if (++s == (uint32_t)C::SP) { s = 0; ph ^= 1; }
-        }
-        if (!ok) break;
-        mma_commit(&acc_full[2 * j + b]);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts_lead(d_tmem, a_tmem + kk * 8,
+                           bdesc + (uint64_t)((kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2), idesc,
+                           (ks != c || kk != 0) ? 1u : 0u, leader);
+        mma_commit_lead(&empty[s], leader);
       }
-      if (!ok) {
-        // let every MMA issued so far finish before TMEM is released
-        mma_commit(&drain[j]);
-        mbar_wait_drain(&drain[j], 0);
+      if (!ok) break;
+      if (nc > 0) {
+        mma_commit_lead(&acc_full[b], leader);
+      } else {                                 // a one-stage K: class 1 has nothing to add
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_full[b]);
       }
+    }
+    if (!ok) {
+      // every MMA issued so far completes before TMEM is released
+      mma_commit_lead(&drain[c], leader);
+      mbar_wait_drain(&drain[c], 0);
     }
     __syncwarp();
   } else if (warp < kEpiWarp0) {
     // ---------------- A dequantisation into TMEM ----------------
-    // Group g takes super-stages g, g + 2, g + 4, ...: it waits once for the
-    // super-stage's raw tiles and its A slots, converts the gq tiles' K
-    // stage (one weight row per thread, in two halves for register
-    // pressure) into TMEM, and signals once.  A super-stage is published
-    // (full barrier) only after the group's next one has been converted up
-    // to its first store, so the store latency overlaps useful work.  This
-    // cannot deadlock: that step waits only for the MMAs to release the slot
-    // of super-stage u + 2 - SP, an earlier one (SP >= 3).
+    // Group c converts the class-c items in order: it loads its row of the
+    // raw tile, converts the first quarter, waits for the A slot, stores it,
+    // converts and stores the other quarters, and signals the item.
     const int q = warp & 3;                          // TMEM lane quarter
-    const int g = (warp - kDQWarp0) >> 2;            // group
+    const int c = (warp - kDQWarp0) >> 2;            // class
     const int row = 32 * q + lane;                   // weight row of the tile
     const uint32_t coff = (uint32_t)row * 16u;       // chunk-major raw tile
     const uint32_t soff = 128u * 64u + (uint32_t)row * 2u;   // INT4 group scale
-    const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + C::A_COL0;
+    const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + C::ACC;
     const uint32_t raw0 = smem_u32(sRaw);
-    constexpr int CPH = F::NC;                       // chunks per half row
-    uint32_t s = 0, ph = 0, r = 0, rph = 0;          // ring positions of super-stage u
-    int pending = -1;                                // A slot whose stores are not yet published
+    constexpr int QC = F::QC;
+    const uint32_t n_items = (uint32_t)(nt * ncls(c));
     bool ok = true;
-    for (int q0 = 0, u = 0; q0 < nt && ok; q0 += G) {
-      const int gq = min(G, nt - q0);
-      for (int ks = 0; ks < KS; ++ks, ++u) {
-        if (u % kGroups == g) {
-          if (!(ok = warp_wait(&raw_full[r], rph, abort_flag))) break;
-          for (int jj = 0; jj < gq; ++jj) {
-            const uint32_t rp = raw0 + (r * G + jj) * C::SLOT;
-            uint4 w0[CPH], w1[CPH];
+    for (uint32_t i = 0; i < n_items; ++i) {
+      const uint32_t r = c * RH + i % RH, rph = (i / RH) & 1;
+      const uint32_t s = c * SH + i % SH, ph = (i / SH) & 1;
+      if (!(ok = warp_wait(&raw_full[r], rph, abort_flag, lim))) break;
+      const uint32_t rp = raw0 + r * C::SLOT;
+      uint4 w[4 * QC];                           // the row's 128 K of codes
 #pragma unroll
-            for (int k = 0; k < CPH; ++k) {
-              asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                           : "=r"(w0[k].x), "=r"(w0[k].y), "=r"(w0[k].z), "=r"(w0[k].w)
-                           : "r"(rp + coff + k * 2048));
-              asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                           : "=r"(w1[k].x), "=r"(w1[k].y), "=r"(w1[k].z), "=r"(w1[k].w)
-                           : "r"(rp + coff + (CPH + k) * 2048));
-            }
-            uint32_t sbits = 0;
-            if constexpr (FMT == QMOE_W_INT4_G128) {
-              unsigned short sv;
-              asm volatile("ld.shared.u16 %0, [%1];" : "=h"(sv) : "r"(rp + soff));
-              sbits = sv;
-            }
-            uint32_t av[kHalf / 2];
-            dequant_slice<FMT>(w0, sbits, av);
-            if (jj == 0) {
-              if (!(ok = warp_wait(&empty[s], ph ^ 1, abort_flag))) break;
-              tc_fence_after();               // TMEM stores after the MMAs' reads of this slot
-              // The previous super-stage's stores were left in flight while
-              // this one was loaded and converted; complete and publish them.
-              if (pending >= 0) {
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&full[pending]);
-              }
-            }
-            const uint32_t ta = tbase + (s * G + jj) * 64;
-#pragma unroll
-            for (int c = 0; c < kHalf / 32; ++c) tmem_st16(ta + 16 * c, &av[16 * c]);
-            dequant_slice<FMT>(w1, sbits, av);
-#pragma unroll
-            for (int c = 0; c < kHalf / 32; ++c) tmem_st16(ta + kHalf / 2 + 16 * c, &av[16 * c]);
-          }
-          if (!ok) break;
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&raw_empty[r]);
-          pending = (int)s;
-        }
-        if (++r == (uint32_t)C::RP) { r = 0; rph ^= 1; }
-        if (++s == (uint32_t)C::SP) { s = 0; ph ^= 1; }
+      for (int k = 0; k < 4 * QC; ++k)
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w[k].x), "=r"(w[k].y), "=r"(w[k].z), "=r"(w[k].w)
+                     : "r"(rp + coff + k * 2048));
+      uint32_t sbits = 0;
+      if constexpr (FMT == QMOE_W_INT4_G128) {
+        unsigned short sv;
+        asm volatile("ld.shared.u16 %0, [%1];" : "=h"(sv) : "r"(rp + soff));
+        sbits = sv;
       }
-    }
-    if (pending >= 0) {
+      // Four quarters of 16 pairs, converted into two alternating register
+      // sets so a conversion never waits for the previous quarter's store to
+      // read its registers.
+      uint32_t av[2][16];
+      dequant_chunks<FMT, QC>(&w[0], sbits, av[0]);
+      if (!(ok = warp_wait(&empty[s], ph ^ 1, abort_flag, lim))) break;
+      tc_fence_after();                          // TMEM stores after the MMAs' reads of this slot
+      const uint32_t ta = tbase + s * 64;
+      tmem_st16(ta, av[0]);
+#pragma unroll
+      for (int qq = 1; qq < 4; ++qq) {
+        dequant_chunks<FMT, QC>(&w[qq * QC], sbits, av[qq & 1]);
+        tmem_st16(ta + 16 * qq, av[qq & 1]);
+      }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&full[pending]);
+      if (lane == 0) {
+        mbar_arrive(&full[s]);
+        mbar_arrive(&raw_empty[r]);
+      }
     }
+    if (!ok) tmem_wait_st();                         // stores issued before the abort land first
   } else {
     // ---------------- epilogue ----------------
     // Each of the 4 epilogue warps owns 32 accumulator rows (TMEM lane
-    // quarter q) and stages and stores its own slice of the output rows, so
-    // only warp-level syncs are needed.  mat 0: 16 intermediate columns
-    // (32 B) per token; mat 1: 32 output columns (64 B) per token.
+    // quarter q), adds the tile's two partials (class 0 + class 1), and
+    // stages and stores its own slice of the output rows, so only warp-level
+    // syncs are needed.  mat 0: 16 intermediate columns (32 B) per token;
+    // mat 1: 32 output columns (64 B) per token.
     const int q = warp & 3;
     const int r = 32 * q + lane;             // accumulator row = tile weight row
     constexpr int WCOLS = MAT == 0 ? 16 : 32;
-    uint16_t* stg = reinterpret_cast<uint16_t*>(sStg) + (size_t)q * BN * WCOLS;
+    constexpr int NCH = BN <= 32 ? BN / 16 : 1;   // 16-column chunks held in registers at once
+    uint16_t* stg = reinterpret_cast<uint16_t*>(sStg) + (size_t)q * 16 * NCH * WCOLS;   // [16 * NCH tokens][WCOLS]
+    const bool two = KS > 1;                 // class 1 received K stages
     bool ok = true;
-    for (int q0 = 0, grp = 0; q0 < nt && ok; q0 += G, ++grp) {
-      const int gq = min(G, nt - q0);
-      const int b = grp & 1;
-      for (int j = 0; j < gq && ok; ++j) {
-        const Tile t = tile_of(q0 + j);
-        const ExpertDev& ex = a.experts[t.seg];
-        const float scale = (FMT != QMOE_W_INT4_G128) ? ex.spc[MAT][t.mb * 128 + r] : 1.0f;
-        ok = warp_wait_backoff(&acc_full[2 * j + b], (grp >> 1) & 1, abort_flag, kSleepEpi);
-        if (!ok) break;
-        tc_fence_after();
-        const int n_mma = max(16, (t.nvalid + 15) & ~15);
-        const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)((2 * j + b) * BN);
-        for (int c0 = 0; c0 < n_mma; c0 += 16) {
-          uint32_t v[16];
-          tmem_ld16(taddr + c0, v);
-          tmem_wait_ld();
-          if (MAT == 0) {
+    for (int tq = 0; tq < nt && ok; ++tq) {
+      const Tile t = tile_of(tq);
+      const ExpertDev& ex = a.experts[t.seg];
+      const float scale = (FMT != QMOE_W_INT4_G128) ? ex.spc[MAT][t.mb * 128 + r] : 1.0f;
+      const int b = NBUF == 2 ? (tq & 1) : 0;
+      const int use = NBUF == 2 ? (tq >> 1) : tq;
+      ok = warp_wait_backoff(&acc_full[b], use & 1, abort_flag, kSleepEpi, lim);
+      if (!ok) break;
+      tc_fence_after();
+      const int n_mma = max(16, (t.nvalid + 15) & ~15);
+      const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * kCls * BN);
+      // Columns [c0, c0 + 16 * NCH) of partial 0 + partial 1, then the output
+      // for them.  For token blocks of up to 32 rows every column is read
+      // before the set is released, so the issuers can start the tile after
+      // next while this one is finished.
+      for (int c0 = 0; c0 < n_mma; c0 += 16 * NCH) {
+        float v[NCH][16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float f = __uint_as_float(v[i]) * scale;
-              const float o = __shfl_xor_sync(0xffffffffu, f, 1);   // up value of the same index
-              if ((lane & 1) == 0) {
-                const float hv = silu_f(f) * o;   // H is fp16 in the fp16 MMA mode, else bf16
-                stg[(c0 + i) * WCOLS + (lane >> 1)] = FMT == kFmtFp8F16 ? f2h(hv) : f2bf(hv);
-              }
+        for (int ch = 0; ch < NCH; ++ch) {
+          if (c0 + 16 * ch < n_mma) {
+            const uint32_t col = taddr + c0 + 16 * ch;
+            uint32_t x0[16], x1[16];
+            tmem_ld16(col, x0);
+            if (two) tmem_ld16(col + BN, x1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              v[ch][i] = (two ? __uint_as_float(x0[i]) + __uint_as_float(x1[i]) : __uint_as_float(x0[i])) * scale;
+          }
+        }
+        if (c0 + 16 * NCH >= n_mma) {             // last columns read: release the set
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[b]);
+        }
+#pragma unroll
+        for (int ch = 0; ch < NCH; ++ch) {
+          const int cc = c0 + 16 * ch;
+          if (cc >= n_mma) break;
+          if (MAT == 0) {
+            // Lanes 2i (gate row) and 2i+1 (up row) share the SwiGLU of
+            // intermediate index i: the even lane produces columns 0-7 of the
+            // chunk, the odd lane columns 8-15.
+            const bool odd = lane & 1;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float send = odd ? v[ch][i] : v[ch][i + 8];
+              const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+              const float hv = odd ? swiglu_f(recv, v[ch][i + 8]) : swiglu_f(v[ch][i], recv);
+              const int col = 16 * ch + i + (odd ? 8 : 0);
+              // H is fp16 in the fp16 MMA mode, else bf16
+              stg[col * WCOLS + (lane >> 1)] = FMT == kFmtFp8F16 ? f2h(hv) : f2bf(hv);
             }
           } else {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) stg[(c0 + i) * WCOLS + lane] = f2bf(__uint_as_float(v[i]) * scale);
+            for (int i = 0; i < 16; ++i) stg[(16 * ch + i) * WCOLS + lane] = f2bf(v[ch][i]);
           }
         }
-        tc_fence_before();
+        // this warp's slice of the staged tokens, coalesced 16-byte stores
         __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[2 * j + b]);
-        constexpr int VPR = WCOLS / 8;         // 16-byte vectors per token row slice
+        constexpr int VPR = WCOLS / 8;       // 16-byte vectors per token row slice
         const int col0 = MAT == 0 ? t.mb * 64 + q * 16 : t.mb * 128 + q * 32;
-        for (int v = lane; v < t.nvalid * VPR; v += 32) {
-          const int n = v / VPR, c = v % VPR;
-          *reinterpret_cast<uint4*>(a.out + (size_t)(t.row0 + n) * a.out_ld + col0 + c * 8) =
-              *reinterpret_cast<const uint4*>(stg + n * WCOLS + c * 8);
+        const int nrows = min(16 * NCH, t.nvalid - c0);
+        for (int v = lane; v < nrows * VPR; v += 32) {
+          const int n = v / VPR, cv = v % VPR;
+          *reinterpret_cast<uint4*>(a.out + (size_t)(t.row0 + c0 + n) * a.out_ld + col0 + cv * 8) =
+              *reinterpret_cast<const uint4*>(stg + n * WCOLS + cv * 8);
         }
         __syncwarp();
       }

@@ -55,7 +55,11 @@ struct GemmArgs {
   uint16_t* out;              // H [P][I] or Y [P][d]
   int out_ld;
   int* err;                   // device error word
+  long long wait_limit;       // SM cycles a bounded wait may last before the kernel aborts
 };
+
+// Default bound of every mbarrier wait in the grouped GEMMs (about a second).
+constexpr long long kWaitLimit = 1ll << 31;
 
 // ---------------------------------------------------------------------------
 // PTX wrappers
@@ -109,14 +113,15 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar_addr, uint32_t 
 }
 
 // Slow path of mbar_wait: sleep-wait with a bound.  Gives up (returns false)
-// when *abort is raised by another role or after ~2^31 SM cycles (about a
-// second), in which case it raises *abort itself.
-static __device__ __noinline__ bool mbar_wait_slow(uint32_t addr, uint32_t parity, volatile int* abort) {
+// when *abort is raised by another role or after `limit` SM cycles, in which
+// case it raises *abort itself.
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t addr, uint32_t parity, volatile int* abort,
+                                                   long long limit) {
   const long long t0 = clock64();
   for (;;) {
     if (mbar_try_wait_sleep(addr, parity)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > (1ll << 31)) {
+    if (clock64() - t0 > limit) {
       *abort = 1;
       return false;
     }
@@ -124,32 +129,33 @@ static __device__ __noinline__ bool mbar_wait_slow(uint32_t addr, uint32_t parit
 }
 
 // Bounded wait for the phase with the given parity (fast path inline).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, long long limit) {
   const uint32_t addr = smem_u32(bar);
   if (mbar_try_wait(addr, parity)) return true;
-  return mbar_wait_slow(addr, parity, abort);
+  return mbar_wait_slow(addr, parity, abort, limit);
 }
 
 // Bounded wait that sleeps ns nanoseconds between polls: for roles whose
 // waits are long and off the critical path, so that their polling leaves the
 // issue slots to the warps doing the work.
 static __device__ __noinline__ bool mbar_wait_backoff_slow(uint32_t addr, uint32_t parity, volatile int* abort,
-                                                           uint32_t ns) {
+                                                           uint32_t ns, long long limit) {
   const long long t0 = clock64();
   for (;;) {
     if (mbar_try_wait(addr, parity)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > (1ll << 31)) {
+    if (clock64() - t0 > limit) {
       *abort = 1;
       return false;
     }
     __nanosleep(ns);
   }
 }
-__device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t ns) {
+__device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t ns,
+                                                  long long limit) {
   const uint32_t addr = smem_u32(bar);
   if (mbar_try_wait(addr, parity)) return true;
-  return mbar_wait_backoff_slow(addr, parity, abort, ns);
+  return mbar_wait_backoff_slow(addr, parity, abort, ns, limit);
 }
 
 // Same, ignoring the abort flag (used while draining on the way out).
@@ -224,6 +230,29 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// The same MMA and commit for a warp that executes the call together
+// (warp-uniform control flow, so the operands stay warp-uniform): only the
+// lane with leader != 0 issues.  A commit tracks the MMAs of the thread that
+// issues it, so one fixed lane issues both.
+__device__ __forceinline__ void mma_bf16_ts_lead(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate, uint32_t leader) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 e, %5, 0;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(leader)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit_lead(uint64_t* bar, uint32_t leader) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "setp.ne.b32 e, %1, 0;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar)),
+      "r"(leader)
       : "memory");
 }
 
