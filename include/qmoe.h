@@ -142,6 +142,17 @@ qmoe_status qmoe_forward_host(qmoe_handle* h, const uint16_t* x_host, int32_t T,
  * the flag.  Returns QMOE_OK otherwise. */
 qmoe_status qmoe_check_error(qmoe_handle* h, void* stream);
 
+/* Bound, in SM clock cycles, of every barrier wait inside the grouped GEMM
+ * kernels of this handle (0 restores the default of 2^31, about a second).
+ * A kernel whose wait runs out stops cleanly: it lets the copies and MMAs it
+ * issued finish, frees its tensor memory and raises the handle's error word,
+ * which qmoe_check_error reports as QMOE_ERR_TIMEOUT; its output is then
+ * undefined.  A limit far below a kernel's normal waits (a few thousand
+ * cycles) makes that path run on purpose, which is how failure detection is
+ * tested; the next forward at the default limit is unaffected.  Takes effect
+ * for forwards enqueued after the call.  cycles < 0 -> QMOE_ERR_INVALID. */
+qmoe_status qmoe_set_wait_limit(qmoe_handle* h, int64_t cycles);
+
 /* Per-kernel timing.  With enable != 0, later qmoe_forward calls record a
  * CUDA event pair around each launch on the caller's stream.
  * qmoe_profile_read synchronises, adds the elapsed milliseconds of every

@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -21,7 +22,7 @@ namespace {
 // Programmatic dependent launch of the kernels after the router.  Off: with
 // it on, the mixed-format workload hit an unspecified launch failure whose
 // cause was not found; every kernel still calls pdl_wait(), a no-op here.
-constexpr bool kUsePdl = false;
+constexpr bool kUsePdl = true;
 
 thread_local std::string g_last_error;
 
@@ -65,16 +66,18 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Row-major bf16 matrix [rows][cols] read in boxes of 64 columns x box_rows
-// rows into 128-byte-swizzled shared memory (rows past the end read as zero).
+// Row-major bf16 matrix [rows][cols] seen as 3-D (64 columns, rows, cols / 64
+// column chunks) and read in boxes of 64 columns x box_rows rows x 2 chunks
+// (one 128-column K stage) into 128-byte-swizzled shared memory laid out
+// [chunk][row][64]; rows past the end read as zero.
 bool encode_rows_map(CUtensorMap* m, const void* base, int rows, int cols, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
-  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  const cuuint64_t dims[3] = {64, (cuuint64_t)rows, (cuuint64_t)cols / 64};
+  const cuuint64_t strides[2] = {(cuuint64_t)cols * 2, 128};
+  const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -102,7 +105,8 @@ struct qmoe_handle {
   float *gates = nullptr, *zpart = nullptr;
   uint16_t *Xp = nullptr, *H = nullptr, *Y = nullptr, *x_stage = nullptr, *out_stage = nullptr;
   int* err = nullptr;
-  int zpart_split_max = 1;
+  int* tile_done = nullptr;              // router: per-32-token-tile completion counters (zero between calls)
+  size_t zpart_floats = 0;               // capacity of the router's partial-logit buffer
   long long wait_limit = kWaitLimit;     // bound of the grouped GEMMs' mbarrier waits (SM cycles)
   // profiling
   bool profiling = false;
@@ -195,9 +199,9 @@ qmoe_status route_impl(qmoe_handle* h, const uint16_t* x, const float* logits, i
     StageTimer tm(h, s, QMOE_STAGE_ROUTER);
     if (x) {
       int split = router_split(T, c.d, c.E, h->num_sms);
-      if (split > h->zpart_split_max) split = h->zpart_split_max;
-      QMOE_CUDA(launch_router(x, h->router_w, h->router_b, T, c.d, c.E, c.k, split, h->zpart, idx,
-                              gates, s),
+      while (split > 1 && (size_t)split * T * c.E > h->zpart_floats) split >>= 1;
+      QMOE_CUDA(launch_router_fused(x, h->router_w, h->router_b, T, c.d, c.E, c.k, split, h->zpart, h->tile_done,
+                                    idx, gates, s),
                 "router launch");
     } else {
       QMOE_CUDA(launch_router_topk(logits, T, c.E, c.k, idx, gates, s), "router top-k launch");
@@ -314,7 +318,6 @@ qmoe_status qmoe_create(const qmoe_config* cfg, const float* router_w, const flo
     return bail(cuda_fail(cudaGetLastError(), "copy expert table"));
 
   // workspace
-  h->zpart_split_max = 16;
   const int n_seg = nexp;
   if ((st = h->alloc(&h->idx, Tm * c.k, "idx")) != QMOE_OK) return bail(st);
   if ((st = h->alloc(&h->gates, Tm * c.k, "gates")) != QMOE_OK) return bail(st);
@@ -337,8 +340,14 @@ qmoe_status qmoe_create(const qmoe_config* cfg, const float* router_w, const flo
   }
   if ((st = h->alloc(&h->sched_scratch, schedule_scratch_ints(c.max_tokens, c.E), "schedule scratch")) != QMOE_OK)
     return bail(st);
-  if ((st = h->alloc(&h->zpart, (size_t)h->zpart_split_max * Tm * c.E, "router partials")) != QMOE_OK)
-    return bail(st);
+  // The router splits d into slices only while its grid of 32 x 32 tiles is
+  // short of the SMs, so split * T * E stays below SMs * 1024 when split > 1;
+  // with one slice the buffer holds the T x E logits themselves.
+  h->zpart_floats = std::max(Tm * (size_t)c.E, (size_t)sms * 1024);
+  if ((st = h->alloc(&h->zpart, h->zpart_floats, "router partials")) != QMOE_OK) return bail(st);
+  if ((st = h->alloc(&h->tile_done, (Tm + 31) / 32, "router tile counters")) != QMOE_OK) return bail(st);
+  if (cudaMemset(h->tile_done, 0, sizeof(int) * ((Tm + 31) / 32)) != cudaSuccess)
+    return bail(cuda_fail(cudaGetLastError(), "memset"));
   if ((st = h->alloc(&h->Xp, P * c.d, "permuted x")) != QMOE_OK) return bail(st);
   if ((st = h->alloc(&h->H, P * c.I, "H")) != QMOE_OK) return bail(st);
   for (int b = 0; b < kNumBn; ++b) {
@@ -450,6 +459,13 @@ qmoe_status qmoe_check_error(qmoe_handle* h, void* stream) {
   return QMOE_OK;
 }
 
+qmoe_status qmoe_set_wait_limit(qmoe_handle* h, int64_t cycles) {
+  if (!h) return fail(QMOE_ERR_INVALID, "handle is NULL");
+  if (cycles < 0) return fail(QMOE_ERR_INVALID, "cycles must be >= 0");
+  h->wait_limit = cycles == 0 ? kWaitLimit : (long long)cycles;
+  return QMOE_OK;
+}
+
 qmoe_status qmoe_profile(qmoe_handle* h, int32_t enable) {
   if (!h) return fail(QMOE_ERR_INVALID, "handle is NULL");
   h->profiling = enable != 0;
@@ -476,7 +492,7 @@ int32_t qmoe_launches_per_forward(const qmoe_handle* h, int32_t T) {
   if (!h) return 0;
   int fmts = 0;
   for (int f = 1; f <= 3; ++f) fmts += h->fmt_present[f] ? 1 : 0;
-  return 5 + 2 * fmts;  // router logits + top-k, schedule, row permutation, gate/up and down per format, combine
+  return 4 + 2 * fmts;  // router, schedule, row permutation, gate/up and down per format, combine
 }
 
 qmoe_status qmoe_destroy(qmoe_handle* h) {

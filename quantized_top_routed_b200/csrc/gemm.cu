@@ -34,22 +34,31 @@
 // Persistent CTAs (one per SM) walk the tile list (segment, 128-row weight
 // block, BN-row token block) built on the device by the schedule kernel;
 // one launch handles the experts of one weight format.  Everything a class
-// touches is private to it: dequantisation group c, issuer c, partial c, and
-// half of the raw ring and of the stage ring (A in TMEM, B in shared memory).
-// So every ring slot has one producer and one consumer that both walk its
-// uses in order, and a parity wait can never be two phases behind.
+// touches is private to it: raw producer c, dequantisation group c, issuer
+// c, partial c, and its own raw ring, A ring (TMEM) and B ring (shared
+// memory).  So every ring slot has one producer and one consumer that both
+// walk its uses in order, and a parity wait can never be two phases behind.
+//
+// Copy requests.  A TMA request holds the warp that issues it for several
+// hundred cycles whatever its size (up to ~16 KB), while requests from
+// different warps proceed in parallel.  So each class has its own producer
+// warp, requests are large (the weight repack stores each class's stages of
+// a block contiguously and one bulk copy brings NST of them; each K stage of
+// B is one 3-D tensor box of 64 columns x BN rows x 2 column chunks), and the
+// issuer warps issue nothing but MMAs.
 // Warp roles, all synchronised through mbarriers:
-//   warp 0       : TMEM allocation; lane 0 streams raw weight tiles (bulk copy)
-//   warp 1       : lane 0 issues the B tile loads (TMA)
-//   warps 2, 3   : MMA issuers of classes 0 and 1 (warp-uniform loops, lane 0 issues)
+//   warps 0, 1   : producer of class 0 / 1 (lane 0): raw weight chunks (bulk
+//                  copies) and B stages (TMA); warp 0 also allocates TMEM
+//   warps 2, 3   : MMA issuer of class 0 / 1 (warp-uniform loops, one
+//                  elected lane issues)
 //   warps 4..11  : dequantise A into TMEM, group c = warps 4 + 4c .. 7 + 4c;
 //                  warp w owns TMEM lane quarter w % 4, one weight row per thread
 //   warps 12..15 : epilogue (TMEM -> registers -> sum of partials, scales,
 //                  SwiGLU -> bf16)
 // Every wait is bounded (GemmArgs::wait_limit cycles): a role that waits too
-// long raises an abort flag, all roles drain what they issued (the producers
-// on barriers that only their own copies complete, the issuers on a commit),
-// TMEM is freed and the error word is set.
+// long raises an abort flag, all roles drain what they issued (copies on
+// barriers that only their own bytes complete, MMAs on a commit), TMEM is
+// freed and the error word is set.
 #include <cuda.h>
 #include <cuda_fp16.h>
 
@@ -58,7 +67,7 @@
 namespace qmoe {
 namespace {
 
-constexpr int kRawWarp = 0, kBWarp = 1, kMmaWarp0 = 2;
+constexpr int kProdWarp0 = 0, kMmaWarp0 = 2;  // producers: warps 0, 1
 constexpr int kCls = 2;                        // stage classes (issuer warp + dequantisation group each)
 constexpr int kDQWarp0 = kMmaWarp0 + kCls;     // first dequantisation warp
 constexpr int kEpiWarp0 = kDQWarp0 + 4 * kCls;
@@ -74,6 +83,7 @@ template <int FMT>
 struct FmtCfg {
   static constexpr int SB = FMT == QMOE_W_INT4_G128 ? 128 * 64 + 256 : 128 * 128;  // bytes of a raw tile
   static constexpr int QC = FMT == QMOE_W_INT4_G128 ? 1 : 2;    // 16-byte chunks per quarter row (16 pairs)
+  static constexpr int NST = FMT == QMOE_W_INT4_G128 ? 2 : 1;   // stages per raw bulk copy (16.5 or 16 KB)
 };
 
 template <int BN, int FMT>
@@ -81,27 +91,34 @@ struct Cfg {
   static constexpr int NBUF = BN <= 32 ? 2 : 1;                      // accumulator sets (double buffer)
   static constexpr int ACC = NBUF * kCls * BN;                       // TMEM columns of the accumulators
   static constexpr int SH0 = ((int)kTmemCols - ACC) / 64 / kCls;
-  static constexpr int SH = SH0 > 3 ? 3 : SH0;                       // stage slots per class
-  static constexpr int SA = kCls * SH;                               // stage ring: A (TMEM) + B (smem)
+  static constexpr int SH = SH0 > 3 ? 3 : SH0;                       // A slots (TMEM) per class
+  static constexpr int SA = kCls * SH;
   static constexpr int B_STAGE = BN * 256;                           // BN rows x 128 K bf16
+  // B stages come from L2 with a TMA round trip of their own, so the B ring
+  // runs deeper than the A ring (which TMEM bounds) where shared memory allows.
+  static constexpr int SHB0 = 96 * 1024 / B_STAGE / kCls;
+  static constexpr int SHB = SHB0 > 8 ? 8 : (SHB0 < 2 ? 2 : SHB0);   // B slots per class
+  static constexpr int SB = kCls * SHB;
   static constexpr int STAGING = 4 * 16 * (BN <= 32 ? BN / 16 : 1) * 64;   // epilogue staging (4 warps)
-  static constexpr int SLOT = (FmtCfg<FMT>::SB + 127) & ~127;        // raw ring slot
-  static constexpr int FIXED = SA * B_STAGE + STAGING + 6 * 1024;
-  static constexpr int R0 = (224 * 1024 - FIXED) / SLOT / kCls;
+  static constexpr int NST = FmtCfg<FMT>::NST;
+  static constexpr int CHUNK = NST * FmtCfg<FMT>::SB;                // raw ring slot
+  static constexpr int FIXED = SB * B_STAGE + STAGING + 6 * 1024;
+  static constexpr int R0 = (224 * 1024 - FIXED) / CHUNK / kCls;
   static constexpr int RH = R0 > 8 ? 8 : R0;                         // raw slots per class
   static constexpr int R = kCls * RH;
   static constexpr int OFF_B = 0;
-  static constexpr int OFF_RAW = OFF_B + SA * B_STAGE;
-  static constexpr int OFF_STG = OFF_RAW + R * SLOT;
-  static constexpr int OFF_TAB = OFF_STG + STAGING;
+  static constexpr int OFF_RAW = OFF_B + SB * B_STAGE;
+  static constexpr int OFF_STG = OFF_RAW + R * CHUNK;
+  static constexpr int OFF_TAB = (OFF_STG + STAGING + 127) & ~127;
   static constexpr int OFF_BAR = (OFF_TAB + 3 * kTabMax * 4 + 127) & ~127;
-  static constexpr int NUM_BARS = 3 * SA + 2 * R + 2 * NBUF + kCls;
+  static constexpr int NUM_BARS = 2 * SA + 2 * SB + 2 * R + 2 * NBUF + kCls;
   static constexpr int OFF_MISC = (OFF_BAR + NUM_BARS * 8 + 15) & ~15;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;                  // + alignment slack
   static_assert(RH >= 2 && SH >= 2, "rings too shallow");
   static_assert(ACC + SA * 64 <= (int)kTmemCols, "TMEM budget");
   static_assert(SMEM <= 232448, "shared memory budget");
-  static_assert(B_STAGE % 1024 == 0 && OFF_RAW % 1024 == 0 && OFF_BAR % 8 == 0 && OFF_MISC % 16 == 0,
+  static_assert(B_STAGE % 1024 == 0 && OFF_RAW % 1024 == 0 && CHUNK % 16 == 0 && OFF_BAR % 8 == 0 &&
+                    OFF_MISC % 16 == 0,
                 "alignment");
 };
 
@@ -221,13 +238,14 @@ __device__ __forceinline__ uint16_t f2h(float f) {
   return *reinterpret_cast<const uint16_t*>(&h);
 }
 
-// TMA: a box of 64 bf16 columns x BN rows of a row-major matrix into
-// 128-byte-swizzled shared memory (rows past the matrix read as zero).
-__device__ __forceinline__ void tma_tile2d(uint32_t dst, const CUtensorMap* map, int col, int row, uint64_t* bar) {
+// TMA: a 3-D box (64 columns x BN rows x 2 column chunks = one K stage of B)
+// of a row-major matrix viewed as (64, rows, cols / 64) into 128-byte-swizzled
+// shared memory laid out [chunk][row][64] (rows past the matrix read as zero).
+__device__ __forceinline__ void tma_tile3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(row), "r"(smem_u32(bar))
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
       : "memory");
 }
 
@@ -246,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap act_map) {
   using C = Cfg<BN, FMT>;
   using F = FmtCfg<FMT>;
-  constexpr int SH = C::SH, RH = C::RH, NBUF = C::NBUF;
+  constexpr int SH = C::SH, SHB = C::SHB, RH = C::RH, NBUF = C::NBUF, NST = C::NST;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sB = smem + C::OFF_B;
@@ -257,9 +275,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   int32_t* s_seg_cnt = s_seg_off + kTabMax;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* full = bars;                      // [SA] A of the item in TMEM (one arrival per dequant warp)
-  uint64_t* bfull = full + C::SA;             // [SA] B tiles of the item landed (TMA bytes only)
-  uint64_t* empty = bfull + C::SA;            // [SA] MMAs done with the slot
-  uint64_t* raw_full = empty + C::SA;         // [R] raw tile of the item landed
+  uint64_t* empty = full + C::SA;             // [SA] MMAs done with the A slot
+  uint64_t* bfull = empty + C::SA;            // [SB] B stage of the item landed (TMA bytes only)
+  uint64_t* bempty = bfull + C::SB;           // [SB] MMAs done with the B slot
+  uint64_t* raw_full = bempty + C::SB;        // [R] raw tile of the item landed
   uint64_t* raw_empty = raw_full + C::R;      // [R] raw tile consumed
   uint64_t* acc_full = raw_empty + C::R;      // [NBUF] both partials of the tile complete
   uint64_t* acc_empty = acc_full + NBUF;      // [NBUF] the epilogue has read the partials
@@ -271,16 +290,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_seg = a.n_seg;
   const int KS = a.K / kBK;
   const long long lim = a.wait_limit;
-  // Items of a class: stage ks of the CTA's tile q with ks = c (mod 2) has
-  // class index q * ncls(c) + ks / 2; it uses stage slot c * SH + index % SH
-  // and raw slot c * RH + index % RH.
+  // Items of a class: stage ks of the CTA's tile q with ks = c (mod 2) is
+  // class stage j = ks / 2 of the tile and has class index i = q * ncls(c) + j;
+  // it uses A slot c * SH + i % SH and B slot c * SHB + i % SHB.  Its raw
+  // codes arrive in chunk g = q * nchunk(c) + j / NST (NST consecutive class
+  // stages, one bulk copy), raw slot c * RH + g % RH.
   auto ncls = [&](int c) { return (KS + 1 - c) >> 1; };
+  auto nchunk = [&](int c) { return (ncls(c) + NST - 1) / NST; };
 
   if (tid == 0) {
     for (int s = 0; s < C::SA; ++s) {
       mbar_init(&full[s], 4);
-      mbar_init(&bfull[s], 1);
       mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < C::SB; ++s) {
+      mbar_init(&bfull[s], 1);
+      mbar_init(&bempty[s], 1);
     }
     for (int r = 0; r < C::R; ++r) {
       mbar_init(&raw_full[r], 1);
@@ -294,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == kRawWarp) tmem_alloc(tmem_slot, kTmemCols);
+  if (warp == kProdWarp0) tmem_alloc(tmem_slot, kTmemCols);
   // Everything above is private to the CTA and may overlap the previous
   // kernel's tail; the tile tables and the activations are read only after
   // that kernel has completed.
@@ -316,75 +341,60 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto tile_of = [&](int q) { return decode_tile((int)blockIdx.x + q * (int)gridDim.x, tab_off, s_seg_off,
                                                  s_seg_cnt, n_seg, BN); };
 
-  if (warp == kRawWarp) {
-    // ---------------- raw weight tiles: one bulk copy per item ----------------
+  if (warp < kMmaWarp0) {
+    // ---------------- producer of class c: raw chunks and B stages ----------------
+    // Items in order: the raw chunk when an item starts one (NST class stages
+    // per bulk copy), then the item's B stage (one 3-D tensor box).
+    const int c = warp - kProdWarp0;
+    const int nc = ncls(c), nch = nchunk(c);
+    const int first_pos = c ? ncls(0) : 0;   // position of the class's first stage in a block
     bool ok = true;
-    uint32_t issued[kCls] = {0, 0};
+    uint32_t raw_issued = 0, b_issued = 0;
     for (int q = 0; q < nt && ok; ++q) {
       const Tile t = tile_of(q);
-      const uint8_t* src = a.experts[t.seg].w[MAT] + (size_t)t.mb * KS * F::SB;
-      for (int ks = 0; ks < KS; ++ks) {
-        const int c = ks & 1;
-        const uint32_t i = (uint32_t)(q * ncls(c) + (ks >> 1));
-        const uint32_t r = c * RH + i % RH, ph = (i / RH) & 1;
-        ok = warp_wait_backoff(&raw_empty[r], ph ^ 1, abort_flag, kSleepRaw, lim);
-        if (!ok) break;
+      const uint8_t* src = a.experts[t.seg].w[MAT] + ((size_t)t.mb * KS + first_pos) * F::SB;
+      for (int j = 0; j < nc; ++j) {
+        if (j % NST == 0) {
+          const int m = j / NST;
+          const uint32_t g = (uint32_t)(q * nch + m);
+          const uint32_t r = c * RH + g % RH, ph = (g / RH) & 1;
+          if (!(ok = warp_wait_backoff(&raw_empty[r], ph ^ 1, abort_flag, kSleepRaw, lim))) break;
+          const uint32_t bytes = (uint32_t)(min(NST, nc - m * NST) * F::SB);
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&raw_full[r], bytes);
+            bulk_g2s(sRaw + r * C::CHUNK, src + (size_t)m * NST * F::SB, bytes, &raw_full[r]);
+          }
+          __syncwarp();
+          raw_issued = g + 1;
+        }
+        const uint32_t i = (uint32_t)(q * nc + j);
+        const uint32_t sb = c * SHB + i % SHB, pb = (i / SHB) & 1;
+        if (!(ok = warp_wait_backoff(&bempty[sb], pb ^ 1, abort_flag, kSleepB, lim))) break;
         if (lane == 0) {
-          mbar_arrive_expect_tx(&raw_full[r], (uint32_t)F::SB);
-          bulk_g2s(sRaw + r * C::SLOT, src + (size_t)ks * F::SB, F::SB, &raw_full[r]);
+          mbar_arrive_expect_tx(&bfull[sb], (uint32_t)C::B_STAGE);
+          tma_tile3d(smem_u32(sB + sb * C::B_STAGE), &act_map, 0, t.row0, 2 * (2 * j + c), &bfull[sb]);
         }
         __syncwarp();
-        issued[c] = i + 1;
+        b_issued = i + 1;
       }
     }
-    // copies that may still be in flight complete before the CTA can exit
+    // copies that may still be in flight land before the CTA can exit (each
+    // barrier completes on its own copies' bytes alone)
     if (lane == 0) {
-      for (int c = 0; c < kCls; ++c) {
-        const uint32_t first = issued[c] > (uint32_t)RH ? issued[c] - RH : 0;
-        for (uint32_t i = first; i < issued[c]; ++i) mbar_wait_drain(&raw_full[c * RH + i % RH], (i / RH) & 1);
-      }
-    }
-    __syncwarp();
-  } else if (warp == kBWarp) {
-    // ---------------- B rows: two TMA tiles per item ----------------
-    bool ok = true;
-    uint32_t issued[kCls] = {0, 0};
-    for (int q = 0; q < nt && ok; ++q) {
-      const int row0 = tile_of(q).row0;
-      for (int ks = 0; ks < KS; ++ks) {
-        const int c = ks & 1;
-        const uint32_t i = (uint32_t)(q * ncls(c) + (ks >> 1));
-        const uint32_t s = c * SH + i % SH, ph = (i / SH) & 1;
-        ok = warp_wait_backoff(&empty[s], ph ^ 1, abort_flag, kSleepB, lim);
-        if (!ok) break;
-        if (lane == 0) {
-          const uint32_t dst = smem_u32(sB + s * C::B_STAGE);
-          mbar_arrive_expect_tx(&bfull[s], (uint32_t)C::B_STAGE);
-          tma_tile2d(dst, &act_map, ks * kBK, row0, &bfull[s]);
-          tma_tile2d(dst + BN * 128, &act_map, ks * kBK + 64, row0, &bfull[s]);
-        }
-        __syncwarp();
-        issued[c] = i + 1;
-      }
-    }
-    // bfull completes on the TMA bytes alone, so this drain ends when the
-    // copies have landed, even after an abort
-    if (lane == 0) {
-      for (int c = 0; c < kCls; ++c) {
-        const uint32_t first = issued[c] > (uint32_t)SH ? issued[c] - SH : 0;
-        for (uint32_t i = first; i < issued[c]; ++i) mbar_wait_drain(&bfull[c * SH + i % SH], (i / SH) & 1);
-      }
+      const uint32_t first = raw_issued > (uint32_t)RH ? raw_issued - RH : 0;
+      for (uint32_t g = first; g < raw_issued; ++g) mbar_wait_drain(&raw_full[c * RH + g % RH], (g / RH) & 1);
+      const uint32_t firstb = b_issued > (uint32_t)SHB ? b_issued - SHB : 0;
+      for (uint32_t i = firstb; i < b_issued; ++i) mbar_wait_drain(&bfull[c * SHB + i % SHB], (i / SHB) & 1);
     }
     __syncwarp();
   } else if (warp < kDQWarp0) {
     // ---------------- MMA issuer of class c ----------------
-    // Stages ks = c, c + 2, ... of every tile, accumulated into partial c of
-    // the tile's accumulator set.  The loop runs on the whole warp; lane 0
-    // issues.
+    // Class stages ks = c, c + 2, ... of every tile, accumulated into partial
+    // c of the tile's accumulator set.  The loop runs on the whole warp; one
+    // elected lane issues.
     const int c = warp - kMmaWarp0;
     const uint64_t bdesc0 = smem_desc_sw128(smem_u32(sB));
     const uint32_t a_tmem0 = tmem_base + C::ACC;
-    const uint32_t leader = lane == 0;         // the lane that issues every MMA and commit of this warp
     const int nc = ncls(c);
     bool ok = true;
     for (int q = 0; q < nt && ok; ++q) {
@@ -395,42 +405,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the epilogue has read this set's previous tile
       if (!(ok = warp_wait(&acc_empty[b], (use & 1) ^ 1, abort_flag, lim))) break;
       const uint32_t d_tmem = tmem_base + (uint32_t)((b * kCls + c) * BN);
-      for (int ks = c; ks < KS; ks += 2) {
-        const uint32_t i = (uint32_t)(q * nc + (ks >> 1));
+      for (int j = 0; j < nc; ++j) {
+        const uint32_t i = (uint32_t)(q * nc + j);
         const uint32_t s = c * SH + i % SH, ph = (i / SH) & 1;
-        if (!(ok = warp_wait(&bfull[s], ph, abort_flag, lim))) break;
+        const uint32_t sb = c * SHB + i % SHB, pb = (i / SHB) & 1;
+        if (!(ok = warp_wait(&bfull[sb], pb, abort_flag, lim))) break;
         if (!(ok = warp_wait(&full[s], ph, abort_flag, lim))) break;
         tc_fence_after();
-        // Descriptors of this slot: only the start-address field moves
+        // Descriptors of these slots: only the start-address field moves
         // (16-byte units), so each MMA's operands are one add away.
-        const uint64_t bdesc = bdesc0 + (uint64_t)(s * (C::B_STAGE >> 4));
+        const uint64_t bdesc = bdesc0 + (uint64_t)(sb * (C::B_STAGE >> 4));
         const uint32_t a_tmem = a_tmem0 + s * 64;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts_lead(d_tmem, a_tmem + kk * 8,
-                           bdesc + (uint64_t)((kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2), idesc,
-                           (ks != c || kk != 0) ? 1u : 0u, leader);
-        mma_commit_lead(&empty[s], leader);
+          mma_bf16_ts_elect(d_tmem, a_tmem + kk * 8,
+                            bdesc + (uint64_t)((kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2), idesc,
+                            (j != 0 || kk != 0) ? 1u : 0u);
+        mma_commit_elect(&empty[s]);
+        mma_commit_elect(&bempty[sb]);
       }
       if (!ok) break;
       if (nc > 0) {
-        mma_commit_lead(&acc_full[b], leader);
+        mma_commit_elect(&acc_full[b]);
       } else {                                 // a one-stage K: class 1 has nothing to add
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_full[b]);
       }
     }
-    if (!ok) {
-      // every MMA issued so far completes before TMEM is released
-      mma_commit_lead(&drain[c], leader);
-      mbar_wait_drain(&drain[c], 0);
-    }
+    // Every MMA this warp issued completes before TMEM is released: after an
+    // abort the epilogue may not have waited for the last ones.
+    mma_commit_elect(&drain[c]);
+    mbar_wait_drain(&drain[c], 0);
     __syncwarp();
   } else if (warp < kEpiWarp0) {
     // ---------------- A dequantisation into TMEM ----------------
     // Group c converts the class-c items in order: it loads its row of the
-    // raw tile, converts the first quarter, waits for the A slot, stores it,
-    // converts and stores the other quarters, and signals the item.
+    // stage's raw codes, converts the first quarter, waits for the A slot,
+    // stores it, converts and stores the other quarters, and signals the item
+    // (and frees the raw chunk after its last stage).
     const int q = warp & 3;                          // TMEM lane quarter
     const int c = (warp - kDQWarp0) >> 2;            // class
     const int row = 32 * q + lane;                   // weight row of the tile
@@ -439,13 +451,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + C::ACC;
     const uint32_t raw0 = smem_u32(sRaw);
     constexpr int QC = F::QC;
-    const uint32_t n_items = (uint32_t)(nt * ncls(c));
+    const int nc = ncls(c), nch = nchunk(c);
     bool ok = true;
-    for (uint32_t i = 0; i < n_items; ++i) {
-      const uint32_t r = c * RH + i % RH, rph = (i / RH) & 1;
+    for (int tq = 0; tq < nt && ok; ++tq) {
+     for (int j = 0; j < nc; ++j) {
+      const uint32_t i = (uint32_t)(tq * nc + j);
+      const int m = j / NST, kin = j - m * NST;     // chunk of the class stage and position in it
+      const uint32_t g = (uint32_t)(tq * nch + m);
+      const uint32_t r = c * RH + g % RH, rph = (g / RH) & 1;
       const uint32_t s = c * SH + i % SH, ph = (i / SH) & 1;
       if (!(ok = warp_wait(&raw_full[r], rph, abort_flag, lim))) break;
-      const uint32_t rp = raw0 + r * C::SLOT;
+      const uint32_t rp = raw0 + r * C::CHUNK + kin * F::SB;
       uint4 w[4 * QC];                           // the row's 128 K of codes
 #pragma unroll
       for (int k = 0; k < 4 * QC; ++k)
@@ -477,8 +493,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&full[s]);
-        mbar_arrive(&raw_empty[r]);
+        if (kin == NST - 1 || j == nc - 1) mbar_arrive(&raw_empty[r]);   // last stage of the chunk
       }
+     }
     }
     if (!ok) tmem_wait_st();                         // stores issued before the abort land first
   } else {
@@ -570,7 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kRawWarp) {
+  if (warp == kProdWarp0) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }

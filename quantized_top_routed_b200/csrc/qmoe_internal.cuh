@@ -40,6 +40,12 @@ __host__ __device__ inline int stage_bytes(int fmt) {
   return fmt == QMOE_W_INT4_G128 ? (128 * 64 + 256) : (128 * 128);
 }
 
+// Position of K stage ks among the KS stages of a repacked 128-row block:
+// the even stages first (in order), then the odd ones.
+__host__ __device__ inline int stage_position(int ks, int KS) {
+  return (ks & 1) ? ((KS + 1) >> 1) + (ks >> 1) : (ks >> 1);
+}
+
 // Arguments of the grouped GEMM kernels.
 struct GemmArgs {
   const ExpertDev* experts;   // [n_seg]
@@ -98,28 +104,45 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
   return ok != 0;
 }
 
-// try_wait with a suspend-time hint: the warp sleeps in hardware until the
-// phase completes or about 10 ms pass, so waiting roles take no issue slots.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar_addr, uint32_t parity) {
+// Non-blocking probe of the phase (test_wait never suspends the warp).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar_addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar_addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// try_wait with a suspend-time hint (ns): the warp sleeps in hardware until
+// the phase completes or the hint passes, so waiting roles take no issue slots.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar_addr, uint32_t parity, uint32_t hint_ns) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar_addr), "r"(parity), "r"(10000000u)
+      : "r"(bar_addr), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }
 
 // Slow path of mbar_wait: sleep-wait with a bound.  Gives up (returns false)
 // when *abort is raised by another role or after `limit` SM cycles, in which
-// case it raises *abort itself.
+// case it raises *abort itself.  Each sleep lasts at most about half the
+// bound (in ns, at ~2 cycles per ns), so the bound is checked in time even
+// when it is short.
 static __device__ __noinline__ bool mbar_wait_slow(uint32_t addr, uint32_t parity, volatile int* abort,
                                                    long long limit) {
   const long long t0 = clock64();
+  const long long h = limit / 4;
+  const uint32_t hint = h > 10000000ll ? 10000000u : (h < 64 ? 64u : (uint32_t)h);
   for (;;) {
-    if (mbar_try_wait_sleep(addr, parity)) return true;
+    if (mbar_try_wait_sleep(addr, parity, hint)) return true;
     if (*abort) return false;
     if (clock64() - t0 > limit) {
       *abort = 1;
@@ -128,10 +151,13 @@ static __device__ __noinline__ bool mbar_wait_slow(uint32_t addr, uint32_t parit
   }
 }
 
-// Bounded wait for the phase with the given parity (fast path inline).
+// Bounded wait for the phase with the given parity.  The inline first probe
+// is test_wait, which never suspends: a blocking try_wait may sleep until the
+// phase completes, past any bound, so an incomplete phase always goes to the
+// bounded slow path.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, long long limit) {
   const uint32_t addr = smem_u32(bar);
-  if (mbar_try_wait(addr, parity)) return true;
+  if (mbar_test_wait(addr, parity)) return true;
   return mbar_wait_slow(addr, parity, abort, limit);
 }
 
@@ -142,7 +168,7 @@ static __device__ __noinline__ bool mbar_wait_backoff_slow(uint32_t addr, uint32
                                                            uint32_t ns, long long limit) {
   const long long t0 = clock64();
   for (;;) {
-    if (mbar_try_wait(addr, parity)) return true;
+    if (mbar_test_wait(addr, parity)) return true;
     if (*abort) return false;
     if (clock64() - t0 > limit) {
       *abort = 1;
@@ -154,7 +180,7 @@ static __device__ __noinline__ bool mbar_wait_backoff_slow(uint32_t addr, uint32
 __device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t ns,
                                                   long long limit) {
   const uint32_t addr = smem_u32(bar);
-  if (mbar_try_wait(addr, parity)) return true;
+  if (mbar_test_wait(addr, parity)) return true;
   return mbar_wait_backoff_slow(addr, parity, abort, ns, limit);
 }
 
@@ -234,25 +260,24 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
 }
 
 // The same MMA and commit for a warp that executes the call together
-// (warp-uniform control flow, so the operands stay warp-uniform): only the
-// lane with leader != 0 issues.  A commit tracks the MMAs of the thread that
-// issues it, so one fixed lane issues both.
-__device__ __forceinline__ void mma_bf16_ts_lead(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                                 uint32_t accumulate, uint32_t leader) {
+// (warp-uniform control flow): elect.sync picks the issuing lane.  With all 32
+// lanes active it elects the same lane every time, so a commit tracks the
+// MMAs issued before it by this warp.
+__device__ __forceinline__ void mma_bf16_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                  uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p, e;\n\t"
-      "setp.ne.b32 e, %5, 0;\n\t"
+      "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\t"
+      "elect.sync r|e, 0xffffffff;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(leader)
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-__device__ __forceinline__ void mma_commit_lead(uint64_t* bar, uint32_t leader) {
+__device__ __forceinline__ void mma_commit_elect(uint64_t* bar) {
   asm volatile(
-      "{\n\t.reg .pred e;\n\t"
-      "setp.ne.b32 e, %1, 0;\n\t"
-      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar)),
-      "r"(leader)
+      "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
+      "elect.sync r|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
       : "memory");
 }
 
@@ -329,6 +354,10 @@ cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem
 cudaError_t launch_router(const uint16_t* x, const float* Wr, const float* bias, int T, int d, int E, int k,
                           int split, float* zpart, int32_t* idx, float* gate, cudaStream_t s);
 cudaError_t launch_router_topk(const float* logits, int T, int E, int k, int32_t* idx, float* gate, cudaStream_t s);
+// launch_router in one launch: tile_done holds ceil(T / 32) counters that are
+// zero before the call and are zero again after it.
+cudaError_t launch_router_fused(const uint16_t* x, const float* Wr, const float* bias, int T, int d, int E, int k,
+                                int split, float* zpart, int* tile_done, int32_t* idx, float* gate, cudaStream_t s);
 int router_split(int T, int d, int E, int num_sms);
 
 // Tile tables written by the schedule kernel: for matrix m (0 gate/up, 1

@@ -1,7 +1,9 @@
 // Weight re-layout at create time: the caller's canonical row-major codes
-// become tiles of 128 weight rows x 128 K that the grouped GEMM streams with
-// one bulk copy each.  Tiles of one 128-row block are consecutive in K, so a
-// block's weights are one contiguous range of memory.
+// become tiles of 128 weight rows x 128 K ("stages") that the grouped GEMM
+// streams with bulk copies.  The stages of one 128-row block form one
+// contiguous range of memory, the even K stages first and then the odd ones
+// (the grouped GEMM's two stage classes), so each class's stages of a block
+// are contiguous and several of them arrive with one bulk copy.
 //
 // Row order inside a tile:
 //   gate/up matrix (mat 0): tile row 2j is gate row 64*mb + j, tile row
@@ -40,7 +42,7 @@ __global__ void repack_kernel(int fmt, int mat, const uint8_t* __restrict__ w, c
   const int mb = rg >> 7, r = rg & 127;
   const int KS = K / kBK;
   const int src = src_row_of(mat, mb, r, I);
-  uint8_t* tile = dst + ((size_t)mb * KS + ks) * stage_bytes(fmt);
+  uint8_t* tile = dst + ((size_t)mb * KS + stage_position(ks, KS)) * stage_bytes(fmt);
   if (fmt == QMOE_W_INT4_G128) {
     const uint8_t* s = w + (size_t)src * (K / 2) + ks * 64;
     auto q_at = [&](int kk) -> uint32_t {  // biased code q + 8 of element kk of this stage

@@ -5,12 +5,13 @@
 // top-k routing; "FineRMoE", Sparse Sum Layer: softmax probabilities as
 // mixing weights.)
 //
-// From activations (two launches): router_logits_kernel computes a 32-token
-// x 32-expert tile of fp32 logits over one slice of d (d is split so the grid
-// covers the SMs when T is small), streaming x and Wr through a 3-stage
-// cp.async ring, and writes its partial sums; router_topk_kernel then runs
-// one warp per token, which sums the slices in a fixed order (so the logits
-// are deterministic), adds the bias and takes the top-k.  From supplied
+// From activations: router_logits_kernel computes a 32-token x 32-expert
+// tile of fp32 logits over one slice of d (d is split so the grid covers the
+// SMs when T is small), streaming x and Wr through a 3-stage cp.async ring,
+// and writes its partial sums; then one warp per token sums the slices in a
+// fixed order (so the logits are deterministic), adds the bias and takes the
+// top-k -- in the layer's forward inside the same launch, by the last CTA to
+// finish each token tile, otherwise in router_topk_kernel.  From supplied
 // logits: router_topk_kernel alone, with one slice.
 #include "qmoe_internal.cuh"
 
@@ -101,9 +102,19 @@ __device__ __forceinline__ void cp16(uint32_t dst, const void* src, uint32_t n) 
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
 }
 
+// EPL = 0: partial logits only.  EPL > 0 (ceil(E / 32) rounded up to 1, 2,
+// 4, 8): afterwards the last CTA to finish a 32-token tile (counted in
+// tile_done[tile], which it resets to 0) takes those tokens' top-k itself,
+// summing the slices in the same fixed order as router_topk_kernel, so the
+// two paths give identical results and the second launch is saved.
+template <int EPL>
 __global__ void __launch_bounds__(kRouterThreads) router_logits_kernel(const uint16_t* __restrict__ x,
                                                                       const float* __restrict__ Wr, int T, int d,
-                                                                      int E, int split, float* __restrict__ zpart) {
+                                                                      int E, int split, float* __restrict__ zpart,
+                                                                      int* __restrict__ tile_done,
+                                                                      const float* __restrict__ bias, int k,
+                                                                      int32_t* __restrict__ idx,
+                                                                      float* __restrict__ gate) {
   extern __shared__ __align__(16) uint8_t rsm[];
   uint16_t* xs = reinterpret_cast<uint16_t*>(rsm);                          // [NST][RT][XS]
   float* ws = reinterpret_cast<float*>(rsm + NST * RT * XS * 2);            // [NST][RE][WS]
@@ -174,6 +185,31 @@ __global__ void __launch_bounds__(kRouterThreads) router_logits_kernel(const uin
   if (ta < T && eb < E) zp[(size_t)ta * E + eb] = acc01;
   if (tb < T && ea < E) zp[(size_t)tb * E + ea] = acc10;
   if (tb < T && eb < E) zp[(size_t)tb * E + eb] = acc11;
+  if constexpr (EPL > 0) {
+    __shared__ int s_last;
+    __threadfence();                            // this CTA's partials are visible device-wide
+    __syncthreads();
+    if (tid == 0) {
+      const int contributors = (int)(gridDim.y * gridDim.z);
+      const int before = atomicAdd(&tile_done[tt], 1);
+      s_last = before == contributors - 1;
+      if (s_last) tile_done[tt] = 0;            // every contributor has arrived: ready for the next call
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    const int warp = tid >> 5, lane = tid & 31;
+    for (int i = warp; i < RT; i += kRouterThreads / 32) {
+      const int t = t0 + i;
+      if (t >= T) break;
+      auto logit = [&](int e) {
+        float acc = 0.f;
+        for (int s2 = 0; s2 < split; ++s2) acc += __ldcg(zpart + ((size_t)s2 * T + t) * E + e);
+        return bias ? acc + bias[e] : acc;
+      };
+      topk_token<EPL>(logit, E, k, lane, idx + (size_t)t * k, gate + (size_t)t * k);
+    }
+  }
 }
 
 // One warp per token: logit(e) = sum over slices s (in order) of zpart[s][t][e],
@@ -219,13 +255,38 @@ int router_split(int T, int d, int E, int num_sms) {
 
 cudaError_t launch_router(const uint16_t* x, const float* Wr, const float* bias, int T, int d, int E, int k, int split,
                           float* zpart, int32_t* idx, float* gate, cudaStream_t s) {
-  cudaError_t e = cudaFuncSetAttribute(router_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemRouter);
+  cudaError_t e = cudaFuncSetAttribute(router_logits_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kSmemRouter);
   if (e != cudaSuccess) return e;
   const dim3 grid((T + RT - 1) / RT, (E + RE - 1) / RE, split);
-  e = launch_ex(router_logits_kernel, grid, dim3(kRouterThreads), kSmemRouter, s, false, x, Wr, T, d, E, split,
-                zpart);
+  e = launch_ex(router_logits_kernel<0>, grid, dim3(kRouterThreads), kSmemRouter, s, false, x, Wr, T, d, E, split,
+                zpart, (int*)nullptr, (const float*)nullptr, k, (int32_t*)nullptr, (float*)nullptr);
   if (e != cudaSuccess) return e;
   return launch_topk(zpart, split, bias, T, E, k, idx, gate, s);
+}
+
+namespace {
+template <int EPL>
+cudaError_t launch_fused(const uint16_t* x, const float* Wr, const float* bias, int T, int d, int E, int k, int split,
+                         float* zpart, int* tile_done, int32_t* idx, float* gate, cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(router_logits_kernel<EPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kSmemRouter);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((T + RT - 1) / RT, (E + RE - 1) / RE, split);
+  return launch_ex(router_logits_kernel<EPL>, grid, dim3(kRouterThreads), kSmemRouter, s, false, x, Wr, T, d, E,
+                   split, zpart, tile_done, bias, k, idx, gate);
+}
+}  // namespace
+
+cudaError_t launch_router_fused(const uint16_t* x, const float* Wr, const float* bias, int T, int d, int E, int k,
+                                int split, float* zpart, int* tile_done, int32_t* idx, float* gate, cudaStream_t s) {
+  switch ((E + 31) / 32) {
+    case 1: return launch_fused<1>(x, Wr, bias, T, d, E, k, split, zpart, tile_done, idx, gate, s);
+    case 2: return launch_fused<2>(x, Wr, bias, T, d, E, k, split, zpart, tile_done, idx, gate, s);
+    case 3:
+    case 4: return launch_fused<4>(x, Wr, bias, T, d, E, k, split, zpart, tile_done, idx, gate, s);
+    default: return launch_fused<8>(x, Wr, bias, T, d, E, k, split, zpart, tile_done, idx, gate, s);
+  }
 }
 
 cudaError_t launch_router_topk(const float* logits, int T, int E, int k, int32_t* idx, float* gate, cudaStream_t s) {

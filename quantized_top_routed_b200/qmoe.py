@@ -32,7 +32,7 @@ STAGES = ("router", "schedule", "gate_up", "down", "combine")
 
 EXPORTS = ("qmoe_create", "qmoe_route", "qmoe_forward", "qmoe_forward_host", "qmoe_check_error",
            "qmoe_profile", "qmoe_profile_read", "qmoe_launches_per_forward", "qmoe_destroy",
-           "qmoe_last_error", "qmoe_route_topk_noalloc")
+           "qmoe_last_error", "qmoe_route_topk_noalloc", "qmoe_set_wait_limit")
 
 
 class QmoeError(RuntimeError):
@@ -83,8 +83,10 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.qmoe_last_error.argtypes = []
     lib.qmoe_last_error.restype = ctypes.c_char_p
     lib.qmoe_route_topk_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp]
+    lib.qmoe_set_wait_limit.argtypes = [vp, ctypes.c_int64]
     for name in ("qmoe_create", "qmoe_route", "qmoe_forward", "qmoe_forward_host", "qmoe_check_error",
-                 "qmoe_profile", "qmoe_profile_read", "qmoe_destroy", "qmoe_route_topk_noalloc"):
+                 "qmoe_profile", "qmoe_profile_read", "qmoe_destroy", "qmoe_route_topk_noalloc",
+                 "qmoe_set_wait_limit"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -148,6 +150,11 @@ def qmoe_forward_host(h: int, x_host, T: int, out_host, stream=None):
 
 def qmoe_check_error(h: int, stream=None):
     _check(load().qmoe_check_error(h, _stream(stream)))
+
+
+def qmoe_set_wait_limit(h: int, cycles: int):
+    """Bound (SM cycles) of the grouped GEMMs' barrier waits; 0 = default."""
+    _check(load().qmoe_set_wait_limit(h, cycles))
 
 
 def qmoe_profile(h: int, enable: bool):

@@ -86,6 +86,9 @@ def test_calls_reject_null_handle():
         qmoe.qmoe_route(None, 16, None, 4, 16, 16, 16, 16, 16, 16)
     with pytest.raises(qmoe.QmoeError):
         qmoe.qmoe_check_error(None)
+    with pytest.raises(qmoe.QmoeError) as ei:
+        qmoe.qmoe_set_wait_limit(None, 1000)
+    assert ei.value.status == qmoe.QMOE_ERR_INVALID
 
 
 @pytest.mark.parametrize("T,d,E,k,why", [
