@@ -88,11 +88,22 @@ struct FmtCfg {
 
 template <int BN, int FMT>
 struct Cfg {
+  // Per-stage scaling (INT4 group-128 with token blocks of up to 32 rows):
+  // A holds the exact codes q, each class stage's MMAs write a D slot of
+  // their own, and the epilogue adds s(row, stage) * D into fp32 registers.
+  static constexpr bool PSS = FMT == QMOE_W_INT4_G128 && BN <= 32;
   static constexpr int NBUF = BN <= 32 ? 2 : 1;                      // accumulator sets (double buffer)
-  static constexpr int ACC = NBUF * kCls * BN;                       // TMEM columns of the accumulators
+  static constexpr int DR = PSS ? (BN == 16 ? 4 : 2) : 0;            // D slots per class (per-stage mode)
+  static constexpr int ACC = PSS ? kCls * DR * BN : NBUF * kCls * BN;   // TMEM columns of the accumulators
   static constexpr int SH0 = ((int)kTmemCols - ACC) / 64 / kCls;
   static constexpr int SH = SH0 > 3 ? 3 : SH0;                       // A slots (TMEM) per class
   static constexpr int SA = kCls * SH;
+  // Scale ring of the per-stage mode: slot i % SC of class c holds the fp32
+  // scales of class item i.  SC >= SH + DR: the dequantisation of item
+  // i + SC waits for the MMAs of item i + SC - SH, which waited for the D
+  // slot that the epilogue freed after item i + SC - SH - DR >= i.
+  static constexpr int SC = PSS ? SH + DR : 0;
+  static constexpr int SCB = kCls * SC * 128 * 4;                    // bytes of the scale ring
   static constexpr int B_STAGE = BN * 256;                           // BN rows x 128 K bf16
   // B stages come from L2 with a TMA round trip of their own, so the B ring
   // runs deeper than the A ring (which TMEM bounds) where shared memory allows.
@@ -102,16 +113,17 @@ struct Cfg {
   static constexpr int STAGING = 4 * 16 * (BN <= 32 ? BN / 16 : 1) * 64;   // epilogue staging (4 warps)
   static constexpr int NST = FmtCfg<FMT>::NST;
   static constexpr int CHUNK = NST * FmtCfg<FMT>::SB;                // raw ring slot
-  static constexpr int FIXED = SB * B_STAGE + STAGING + 6 * 1024;
+  static constexpr int FIXED = SB * B_STAGE + STAGING + SCB + 6 * 1024;
   static constexpr int R0 = (224 * 1024 - FIXED) / CHUNK / kCls;
   static constexpr int RH = R0 > 8 ? 8 : R0;                         // raw slots per class
   static constexpr int R = kCls * RH;
   static constexpr int OFF_B = 0;
   static constexpr int OFF_RAW = OFF_B + SB * B_STAGE;
   static constexpr int OFF_STG = OFF_RAW + R * CHUNK;
-  static constexpr int OFF_TAB = (OFF_STG + STAGING + 127) & ~127;
+  static constexpr int OFF_SC = (OFF_STG + STAGING + 127) & ~127;
+  static constexpr int OFF_TAB = (OFF_SC + SCB + 127) & ~127;
   static constexpr int OFF_BAR = (OFF_TAB + 3 * kTabMax * 4 + 127) & ~127;
-  static constexpr int NUM_BARS = 2 * SA + 2 * SB + 2 * R + 2 * NBUF + kCls;
+  static constexpr int NUM_BARS = 2 * SA + 2 * SB + 2 * R + 2 * NBUF + kCls + (PSS ? 2 * kCls * DR + kCls * SC : 0);
   static constexpr int OFF_MISC = (OFF_BAR + NUM_BARS * 8 + 15) & ~15;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;                  // + alignment slack
   static_assert(RH >= 2 && SH >= 2, "rings too shallow");
@@ -168,6 +180,13 @@ __device__ __forceinline__ void deq_int4_word(uint32_t w, uint32_t s2, uint32_t*
     o[j] = bf2_mul(bf2_sub(t, 0x43084308u), s2);                           // (. - 136) * s
   }
 }
+// 8 biased nibbles (q + 8) -> 4 bf16 pairs of q (exact; the group scale is
+// applied to the stage's fp32 result instead).
+__device__ __forceinline__ void deq_int4_word_q(uint32_t w, uint32_t* o) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    o[j] = bf2_sub(lop_and_or(w >> (4 * j), 0x000F000Fu, 0x43004300u), 0x43084308u);   // 136 + q - 136
+}
 // 4 int8 codes (byte order k0 k2 k1 k3) -> 2 bf16 pairs of q (exact).
 __device__ __forceinline__ void deq_int8_word(uint32_t w, uint32_t* o) {
   o[0] = bf2_sub(lop_and_or(w, 0x007F007Fu, 0x43004300u), (w & 0x00800080u) ^ 0x43004300u);
@@ -196,11 +215,16 @@ __device__ __forceinline__ void deq_fp8_f16_word(uint32_t w, uint32_t* o) {
 }
 
 // NCHK of this thread's 16-byte chunks (K order) -> bf16 (or fp16) pairs.
-template <int FMT, int NCHK>
+template <int FMT, int NCHK, bool PSS = false>
 __device__ __forceinline__ void dequant_chunks(const uint4* w, uint32_t sbits, uint32_t* av) {
 #pragma unroll
   for (int c = 0; c < NCHK; ++c) {
-    if constexpr (FMT == QMOE_W_INT4_G128) {
+    if constexpr (PSS) {
+      deq_int4_word_q(w[c].x, &av[16 * c + 0]);
+      deq_int4_word_q(w[c].y, &av[16 * c + 4]);
+      deq_int4_word_q(w[c].z, &av[16 * c + 8]);
+      deq_int4_word_q(w[c].w, &av[16 * c + 12]);
+    } else if constexpr (FMT == QMOE_W_INT4_G128) {
       const uint32_t s2 = sbits | (sbits << 16);
       deq_int4_word(w[c].x, s2, &av[16 * c + 0]);
       deq_int4_word(w[c].y, s2, &av[16 * c + 4]);
@@ -283,6 +307,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_full = raw_empty + C::R;      // [NBUF] both partials of the tile complete
   uint64_t* acc_empty = acc_full + NBUF;      // [NBUF] the epilogue has read the partials
   uint64_t* drain = acc_empty + NBUF;         // [kCls] abort path of the issuers
+  uint64_t* dfull = drain + kCls;             // [kCls * DR] per-stage mode: the stage's D slot is complete
+  uint64_t* dempty = dfull + kCls * C::DR;    // [kCls * DR] per-stage mode: the epilogue has read the D slot
+  uint64_t* scfull = dempty + kCls * C::DR;   // [kCls * SC] per-stage mode: the item's scales are written
+  float* sScale = reinterpret_cast<float*>(smem + C::OFF_SC);   // [kCls][SC][128]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -316,6 +344,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acc_empty[b], 4);     // one arrival per epilogue warp
     }
     for (int c = 0; c < kCls; ++c) mbar_init(&drain[c], 1);
+    for (int d = 0; d < kCls * C::DR; ++d) {
+      mbar_init(&dfull[d], 1);
+      mbar_init(&dempty[d], 4);        // one arrival per epilogue warp
+    }
+    for (int d = 0; d < kCls * C::SC; ++d) mbar_init(&scfull[d], 4);   // one arrival per dequant warp
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -390,7 +423,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp < kDQWarp0) {
     // ---------------- MMA issuer of class c ----------------
     // Class stages ks = c, c + 2, ... of every tile, accumulated into partial
-    // c of the tile's accumulator set.  The loop runs on the whole warp; one
+    // c of the tile's accumulator set (per-stage mode: each stage into the
+    // next D slot of the class).  The loop runs on the whole warp; one
     // elected lane issues.
     const int c = warp - kMmaWarp0;
     const uint64_t bdesc0 = smem_desc_sw128(smem_u32(sB));
@@ -403,12 +437,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b = NBUF == 2 ? (q & 1) : 0;    // accumulator set of this tile
       const int use = NBUF == 2 ? (q >> 1) : q;  // its use count before this tile
       // the epilogue has read this set's previous tile
-      if (!(ok = warp_wait(&acc_empty[b], (use & 1) ^ 1, abort_flag, lim))) break;
-      const uint32_t d_tmem = tmem_base + (uint32_t)((b * kCls + c) * BN);
+      if (!C::PSS && !(ok = warp_wait(&acc_empty[b], (use & 1) ^ 1, abort_flag, lim))) break;
+      uint32_t d_tmem = tmem_base + (uint32_t)((b * kCls + c) * BN);
       for (int j = 0; j < nc; ++j) {
         const uint32_t i = (uint32_t)(q * nc + j);
         const uint32_t s = c * SH + i % SH, ph = (i / SH) & 1;
         const uint32_t sb = c * SHB + i % SHB, pb = (i / SHB) & 1;
+        const uint32_t ds = c * C::DR + (C::PSS ? i % C::DR : 0);
+        if constexpr (C::PSS) {                  // the epilogue has read this D slot's previous stage
+          if (!(ok = warp_wait(&dempty[ds], ((i / C::DR) & 1) ^ 1, abort_flag, lim))) break;
+          d_tmem = tmem_base + ds * BN;
+        }
         if (!(ok = warp_wait(&bfull[sb], pb, abort_flag, lim))) break;
         if (!(ok = warp_wait(&full[s], ph, abort_flag, lim))) break;
         tc_fence_after();
@@ -420,11 +459,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16_ts_elect(d_tmem, a_tmem + kk * 8,
                             bdesc + (uint64_t)((kk >> 2) * (BN * 128 >> 4) + (kk & 3) * 2), idesc,
-                            (j != 0 || kk != 0) ? 1u : 0u);
+                            ((C::PSS ? 0 : j) != 0 || kk != 0) ? 1u : 0u);
         mma_commit_elect(&empty[s]);
         mma_commit_elect(&bempty[sb]);
+        if constexpr (C::PSS) mma_commit_elect(&dfull[ds]);
       }
       if (!ok) break;
+      if constexpr (C::PSS) continue;
       if (nc > 0) {
         mma_commit_elect(&acc_full[b]);
       } else {                                 // a one-stage K: class 1 has nothing to add
@@ -478,20 +519,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       // sets so a conversion never waits for the previous quarter's store to
       // read its registers.
       uint32_t av[2][16];
-      dequant_chunks<FMT, QC>(&w[0], sbits, av[0]);
+      dequant_chunks<FMT, QC, C::PSS>(&w[0], sbits, av[0]);
       if (!(ok = warp_wait(&empty[s], ph ^ 1, abort_flag, lim))) break;
       tc_fence_after();                          // TMEM stores after the MMAs' reads of this slot
       const uint32_t ta = tbase + s * 64;
       tmem_st16(ta, av[0]);
+      const uint32_t scs = (uint32_t)c * C::SC + (C::PSS ? i % C::SC : 0);   // scale slot (per-stage mode)
+      if constexpr (C::PSS) sScale[scs * 128 + row] = __uint_as_float(sbits << 16);
 #pragma unroll
       for (int qq = 1; qq < 4; ++qq) {
-        dequant_chunks<FMT, QC>(&w[qq * QC], sbits, av[qq & 1]);
+        dequant_chunks<FMT, QC, C::PSS>(&w[qq * QC], sbits, av[qq & 1]);
         tmem_st16(ta + 16 * qq, av[qq & 1]);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
+        if constexpr (C::PSS) mbar_arrive(&scfull[scs]);
         mbar_arrive(&full[s]);
         if (kin == NST - 1 || j == nc - 1) mbar_arrive(&raw_empty[r]);   // last stage of the chunk
       }
@@ -512,75 +556,115 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint16_t* stg = reinterpret_cast<uint16_t*>(sStg) + (size_t)q * 16 * NCH * WCOLS;   // [16 * NCH tokens][WCOLS]
     const bool two = KS > 1;                 // class 1 received K stages
     bool ok = true;
+    // Output of columns [c0, c0 + 16 * NCH) of the tile (v: the fp32
+    // accumulator row of this thread for those token columns).
+    auto emit = [&](const Tile& t, int c0, int n_mma, float (&v)[NCH][16]) {
+#pragma unroll
+      for (int ch = 0; ch < NCH; ++ch) {
+        const int cc = c0 + 16 * ch;
+        if (cc >= n_mma) break;
+        if (MAT == 0) {
+          // Lanes 2i (gate row) and 2i+1 (up row) share the SwiGLU of
+          // intermediate index i: the even lane produces columns 0-7 of the
+          // chunk, the odd lane columns 8-15.
+          const bool odd = lane & 1;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float send = odd ? v[ch][i] : v[ch][i + 8];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+            const float hv = odd ? swiglu_f(recv, v[ch][i + 8]) : swiglu_f(v[ch][i], recv);
+            const int col = 16 * ch + i + (odd ? 8 : 0);
+            // H is fp16 in the fp16 MMA mode, else bf16
+            stg[col * WCOLS + (lane >> 1)] = FMT == kFmtFp8F16 ? f2h(hv) : f2bf(hv);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) stg[(16 * ch + i) * WCOLS + lane] = f2bf(v[ch][i]);
+        }
+      }
+      // this warp's slice of the staged tokens, coalesced 16-byte stores
+      __syncwarp();
+      constexpr int VPR = WCOLS / 8;       // 16-byte vectors per token row slice
+      const int col0 = MAT == 0 ? t.mb * 64 + q * 16 : t.mb * 128 + q * 32;
+      const int nrows = min(16 * NCH, t.nvalid - c0);
+      for (int u = lane; u < nrows * VPR; u += 32) {
+        const int n = u / VPR, cv = u % VPR;
+        *reinterpret_cast<uint4*>(a.out + (size_t)(t.row0 + c0 + n) * a.out_ld + col0 + cv * 8) =
+            *reinterpret_cast<const uint4*>(stg + n * WCOLS + cv * 8);
+      }
+      __syncwarp();
+    };
     for (int tq = 0; tq < nt && ok; ++tq) {
       const Tile t = tile_of(tq);
-      const ExpertDev& ex = a.experts[t.seg];
-      const float scale = (FMT != QMOE_W_INT4_G128) ? ex.spc[MAT][t.mb * 128 + r] : 1.0f;
-      const int b = NBUF == 2 ? (tq & 1) : 0;
-      const int use = NBUF == 2 ? (tq >> 1) : tq;
-      ok = warp_wait_backoff(&acc_full[b], use & 1, abort_flag, kSleepEpi, lim);
-      if (!ok) break;
-      tc_fence_after();
       const int n_mma = max(16, (t.nvalid + 15) & ~15);
-      const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * kCls * BN);
-      // Columns [c0, c0 + 16 * NCH) of partial 0 + partial 1, then the output
-      // for them.  For token blocks of up to 32 rows every column is read
-      // before the set is released, so the issuers can start the tile after
-      // next while this one is finished.
-      for (int c0 = 0; c0 < n_mma; c0 += 16 * NCH) {
+      if constexpr (C::PSS) {
+        // Stages in K order (the classes alternate): acc += s(row, stage) * D.
         float v[NCH][16];
 #pragma unroll
-        for (int ch = 0; ch < NCH; ++ch) {
-          if (c0 + 16 * ch < n_mma) {
-            const uint32_t col = taddr + c0 + 16 * ch;
-            uint32_t x0[16], x1[16];
-            tmem_ld16(col, x0);
-            if (two) tmem_ld16(col + BN, x1);
-            tmem_wait_ld();
+        for (int ch = 0; ch < NCH; ++ch)
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              v[ch][i] = (two ? __uint_as_float(x0[i]) + __uint_as_float(x1[i]) : __uint_as_float(x0[i])) * scale;
-          }
-        }
-        if (c0 + 16 * NCH >= n_mma) {             // last columns read: release the set
+          for (int i = 0; i < 16; ++i) v[ch][i] = 0.f;
+        for (int ks = 0; ks < KS; ++ks) {
+          const int c = ks & 1;
+          const uint32_t i = (uint32_t)(tq * ncls(c) + (ks >> 1));
+          const uint32_t ds = c * C::DR + i % C::DR, scs = c * C::SC + i % C::SC;
+          if (!(ok = warp_wait(&dfull[ds], (i / C::DR) & 1, abort_flag, lim))) break;
+          if (!(ok = warp_wait(&scfull[scs], (i / C::SC) & 1, abort_flag, lim))) break;
+          tc_fence_after();
+          const float sc = sScale[scs * 128 + r];
+          const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + ds * BN;
+          uint32_t x[NCH][16];
+#pragma unroll
+          for (int ch = 0; ch < NCH; ++ch)
+            if (16 * ch < n_mma) tmem_ld16(taddr + 16 * ch, x[ch]);
+          tmem_wait_ld();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[b]);
-        }
+          if (lane == 0) mbar_arrive(&dempty[ds]);   // the scale was read above, before the release
 #pragma unroll
-        for (int ch = 0; ch < NCH; ++ch) {
-          const int cc = c0 + 16 * ch;
-          if (cc >= n_mma) break;
-          if (MAT == 0) {
-            // Lanes 2i (gate row) and 2i+1 (up row) share the SwiGLU of
-            // intermediate index i: the even lane produces columns 0-7 of the
-            // chunk, the odd lane columns 8-15.
-            const bool odd = lane & 1;
+          for (int ch = 0; ch < NCH; ++ch)
+            if (16 * ch < n_mma) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float send = odd ? v[ch][i] : v[ch][i + 8];
-              const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-              const float hv = odd ? swiglu_f(recv, v[ch][i + 8]) : swiglu_f(v[ch][i], recv);
-              const int col = 16 * ch + i + (odd ? 8 : 0);
-              // H is fp16 in the fp16 MMA mode, else bf16
-              stg[col * WCOLS + (lane >> 1)] = FMT == kFmtFp8F16 ? f2h(hv) : f2bf(hv);
+              for (int e = 0; e < 16; ++e) v[ch][e] = fmaf(sc, __uint_as_float(x[ch][e]), v[ch][e]);
             }
-          } else {
+        }
+        if (!ok) break;
+        emit(t, 0, n_mma, v);
+      } else {
+        const ExpertDev& ex = a.experts[t.seg];
+        const float scale = (FMT != QMOE_W_INT4_G128) ? ex.spc[MAT][t.mb * 128 + r] : 1.0f;
+        const int b = NBUF == 2 ? (tq & 1) : 0;
+        const int use = NBUF == 2 ? (tq >> 1) : tq;
+        ok = warp_wait_backoff(&acc_full[b], use & 1, abort_flag, kSleepEpi, lim);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * kCls * BN);
+        // Columns [c0, c0 + 16 * NCH) of partial 0 + partial 1, then the output
+        // for them.  For token blocks of up to 32 rows every column is read
+        // before the set is released, so the issuers can start the tile after
+        // next while this one is finished.
+        for (int c0 = 0; c0 < n_mma; c0 += 16 * NCH) {
+          float v[NCH][16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) stg[(16 * ch + i) * WCOLS + lane] = f2bf(v[ch][i]);
+          for (int ch = 0; ch < NCH; ++ch) {
+            if (c0 + 16 * ch < n_mma) {
+              const uint32_t col = taddr + c0 + 16 * ch;
+              uint32_t x0[16], x1[16];
+              tmem_ld16(col, x0);
+              if (two) tmem_ld16(col + BN, x1);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                v[ch][i] = (two ? __uint_as_float(x0[i]) + __uint_as_float(x1[i]) : __uint_as_float(x0[i])) * scale;
+            }
           }
+          if (c0 + 16 * NCH >= n_mma) {             // last columns read: release the set
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[b]);
+          }
+          emit(t, c0, n_mma, v);
         }
-        // this warp's slice of the staged tokens, coalesced 16-byte stores
-        __syncwarp();
-        constexpr int VPR = WCOLS / 8;       // 16-byte vectors per token row slice
-        const int col0 = MAT == 0 ? t.mb * 64 + q * 16 : t.mb * 128 + q * 32;
-        const int nrows = min(16 * NCH, t.nvalid - c0);
-        for (int v = lane; v < nrows * VPR; v += 32) {
-          const int n = v / VPR, cv = v % VPR;
-          *reinterpret_cast<uint4*>(a.out + (size_t)(t.row0 + c0 + n) * a.out_ld + col0 + cv * 8) =
-              *reinterpret_cast<const uint4*>(stg + n * WCOLS + cv * 8);
-        }
-        __syncwarp();
       }
     }
   }

@@ -132,22 +132,24 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar_addr, uint32_t 
 }
 
 // Slow path of mbar_wait: sleep-wait with a bound.  Gives up (returns false)
-// when *abort is raised by another role or after `limit` SM cycles, in which
-// case it raises *abort itself.  Each sleep lasts at most about half the
-// bound (in ns, at ~2 cycles per ns), so the bound is checked in time even
-// when it is short.
+// when *abort is raised by another role or once `limit` SM cycles have
+// passed, in which case it raises *abort itself.  The sleep hint is only a
+// hint (the warp may sleep until the phase completes), so the time is
+// checked after every return of try_wait: a wait that outlived the bound
+// counts as timed out even if its phase completed meanwhile.
 static __device__ __noinline__ bool mbar_wait_slow(uint32_t addr, uint32_t parity, volatile int* abort,
                                                    long long limit) {
   const long long t0 = clock64();
   const long long h = limit / 4;
   const uint32_t hint = h > 10000000ll ? 10000000u : (h < 64 ? 64u : (uint32_t)h);
   for (;;) {
-    if (mbar_try_wait_sleep(addr, parity, hint)) return true;
-    if (*abort) return false;
+    const bool done = mbar_try_wait_sleep(addr, parity, hint);
     if (clock64() - t0 > limit) {
       *abort = 1;
       return false;
     }
+    if (done) return true;
+    if (*abort) return false;
   }
 }
 

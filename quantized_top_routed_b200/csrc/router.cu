@@ -29,73 +29,109 @@ constexpr int WS = RC + 4;      // fp32 row stride of the Wr stage
 constexpr int kRouterThreads = 256;
 constexpr int kSmemPipe = NST * (RT * XS * 2 + RE * WS * 4);
 constexpr int kSmemRouter = kSmemPipe;
+static_assert(kSmemPipe >= RT * kMaxE * 4, "the top-k tail keeps the tile's logits in the pipeline buffers");
 
-// Warp arg-max over (value, index): larger value wins, lower index on ties.
-__device__ __forceinline__ void warp_argmax(float& v, int& e) {
+// One warp: softmax + top-k + renormalisation of the E logits of NT tokens
+// at once (the tokens' shuffle chains interleave; each token's arithmetic is
+// the same as with NT = 1).  logit(u, e) gives the fp32 logit of expert e
+// (bias included) for the warp's token u; token u's outputs go to
+// idx0 + u * ld and gate0 + u * ld when u < nvalid.
+template <int EPL, int NT, class LogitFn>
+__device__ __forceinline__ void topk_tokens(LogitFn logit, int E, int k, int lane, int32_t* idx0, float* gate0,
+                                            size_t ld, int nvalid) {
+  static_assert(NT * EPL <= 32, "one bit per (token, expert slot)");
+  float z[NT][EPL];
+  uint32_t live = 0;                       // bit u * EPL + i: expert lane + 32 i of token u still unpicked
+  float m[NT];
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    const float ov = __shfl_xor_sync(0xffffffffu, v, off);
-    const int oe = __shfl_xor_sync(0xffffffffu, e, off);
-    if (ov > v || (ov == v && oe < e)) {
-      v = ov;
-      e = oe;
-    }
-  }
-}
-
-// One warp: softmax + top-k + renormalisation of one token's E logits.
-// logit(e) gives the fp32 logit of expert e (bias included).
-template <int EPL, class LogitFn>
-__device__ __forceinline__ void topk_token(LogitFn logit, int E, int k, int lane, int32_t* idx_row,
-                                           float* gate_row) {
-  float z[EPL];
-  bool live[EPL];
-  float m = -INFINITY;
-#pragma unroll
-  for (int i = 0; i < EPL; ++i) {
-    const int e = lane + 32 * i;
-    live[i] = e < E;
-    z[i] = live[i] ? logit(e) : -INFINITY;
-    m = fmaxf(m, z[i]);
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-  float den = 0.f;
-#pragma unroll
-  for (int i = 0; i < EPL; ++i)
-    if (live[i]) den += expf(z[i] - m);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
-
-  float my_p = 0.f;
-  int my_e = 0;
-  for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
+  for (int u = 0; u < NT; ++u) {
+    m[u] = -INFINITY;
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
       const int e = lane + 32 * i;
-      if (live[i] && (z[i] > bv || (z[i] == bv && e < be))) {
-        bv = z[i];
-        be = e;
-      }
+      const bool ok = e < E;
+      if (ok) live |= 1u << (u * EPL + i);
+      z[u][i] = ok ? logit(u, e) : -INFINITY;
+      m[u] = fmaxf(m[u], z[u][i]);
     }
-    warp_argmax(bv, be);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+    for (int u = 0; u < NT; ++u) m[u] = fmaxf(m[u], __shfl_xor_sync(0xffffffffu, m[u], off));
+  float den[NT];
+#pragma unroll
+  for (int u = 0; u < NT; ++u) {
+    den[u] = 0.f;
 #pragma unroll
     for (int i = 0; i < EPL; ++i)
-      if (lane + 32 * i == be) live[i] = false;
-    if (lane == j) {
-      my_e = be;
-      my_p = expf(bv - m) / den;
+      if (live >> (u * EPL + i) & 1u) den[u] += expf(z[u][i] - m[u]);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+    for (int u = 0; u < NT; ++u) den[u] += __shfl_xor_sync(0xffffffffu, den[u], off);
+
+  float my_p[NT];
+  int my_e[NT];
+#pragma unroll
+  for (int u = 0; u < NT; ++u) {
+    my_p[u] = 0.f;
+    my_e[u] = 0;
+  }
+  for (int j = 0; j < k; ++j) {
+    float bv[NT];
+    int be[NT];
+#pragma unroll
+    for (int u = 0; u < NT; ++u) {
+      bv[u] = -INFINITY;
+      be[u] = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        if ((live >> (u * EPL + i) & 1u) && (z[u][i] > bv[u] || (z[u][i] == bv[u] && e < be[u]))) {
+          bv[u] = z[u][i];
+          be[u] = e;
+        }
+      }
+    }
+    // warp arg-max: larger value wins, lower index on ties
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+      for (int u = 0; u < NT; ++u) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv[u], off);
+        const int oe = __shfl_xor_sync(0xffffffffu, be[u], off);
+        if (ov > bv[u] || (ov == bv[u] && oe < be[u])) {
+          bv[u] = ov;
+          be[u] = oe;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < NT; ++u) {
+#pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if (lane + 32 * i == be[u]) live &= ~(1u << (u * EPL + i));
+      if (lane == j) {
+        my_e[u] = be[u];
+        my_p[u] = expf(bv[u] - m[u]) / den[u];
+      }
     }
   }
-  float psum = lane < k ? my_p : 0.f;
+  float psum[NT];
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, off);
-  if (lane < k) {
-    idx_row[lane] = my_e;
-    gate_row[lane] = my_p / psum;
-  }
+  for (int u = 0; u < NT; ++u) psum[u] = lane < k ? my_p[u] : 0.f;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+    for (int u = 0; u < NT; ++u) psum[u] += __shfl_xor_sync(0xffffffffu, psum[u], off);
+#pragma unroll
+  for (int u = 0; u < NT; ++u)
+    if (u < nvalid && lane < k) {
+      idx0[u * ld + lane] = my_e[u];
+      gate0[u * ld + lane] = my_p[u] / psum[u];
+    }
 }
 
 __device__ __forceinline__ void cp16(uint32_t dst, const void* src, uint32_t n) {
@@ -198,17 +234,53 @@ __global__ void __launch_bounds__(kRouterThreads) router_logits_kernel(const uin
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    const int warp = tid >> 5, lane = tid & 31;
-    for (int i = warp; i < RT; i += kRouterThreads / 32) {
-      const int t = t0 + i;
-      if (t >= T) break;
-      auto logit = [&](int e) {
-        float acc = 0.f;
-        for (int s2 = 0; s2 < split; ++s2) acc += __ldcg(zpart + ((size_t)s2 * T + t) * E + e);
-        return bias ? acc + bias[e] : acc;
-      };
-      topk_token<EPL>(logit, E, k, lane, idx + (size_t)t * k, gate + (size_t)t * k);
+    // The tile's logits into shared memory (the pipeline buffers are free):
+    // every (token, expert) pair adds its slices in ascending order, with the
+    // loads of four slices of eight pairs in flight together.
+    float* zs = reinterpret_cast<float*>(rsm);   // [nt][E]
+    const int nt = min(RT, T - t0), np = nt * E;
+    const float* zt = zpart + (size_t)t0 * E;
+    const size_t sstride = (size_t)T * E;
+    for (int p0 = 0; p0 < np; p0 += 8 * kRouterThreads) {
+      float acc[8];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) acc[m] = 0.f;
+      int s2 = 0;
+      for (; s2 + 4 <= split; s2 += 4) {
+        float v[4][8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const int p = p0 + m * kRouterThreads + tid;
+            v[u][m] = p < np ? __ldcg(zt + (size_t)(s2 + u) * sstride + p) : 0.f;
+          }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int m = 0; m < 8; ++m) acc[m] += v[u][m];
+      }
+      for (; s2 < split; ++s2)
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const int p = p0 + m * kRouterThreads + tid;
+          if (p < np) acc[m] += __ldcg(zt + (size_t)s2 * sstride + p);
+        }
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const int p = p0 + m * kRouterThreads + tid;
+        if (p < np) zs[p] = bias ? acc[m] + bias[p % E] : acc[m];
+      }
     }
+    __syncthreads();
+    // warp w takes tokens w + 8u (u < 4) of the tile, all four at once
+    constexpr int kWarps = kRouterThreads / 32, NT = RT / kWarps;
+    const int warp = tid >> 5, lane = tid & 31;
+    if (warp >= nt) return;
+    const int nvalid = min(NT, (nt - warp + kWarps - 1) / kWarps);
+    auto logit = [&](int u, int e) { return zs[min(warp + kWarps * u, nt - 1) * E + e]; };
+    topk_tokens<EPL, NT>(logit, E, k, lane, idx + (size_t)(t0 + warp) * k, gate + (size_t)(t0 + warp) * k,
+                         (size_t)kWarps * k, nvalid);
   }
 }
 
@@ -222,12 +294,12 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
   const int t = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
-  auto logit = [&](int e) {
+  auto logit = [&](int, int e) {
     float acc = 0.f;
     for (int s2 = 0; s2 < split; ++s2) acc += __ldcg(zpart + ((size_t)s2 * T + t) * E + e);
     return bias ? acc + bias[e] : acc;
   };
-  topk_token<EPL>(logit, E, k, lane, idx + (size_t)t * k, gate + (size_t)t * k);
+  topk_tokens<EPL, 1>(logit, E, k, lane, idx + (size_t)t * k, gate + (size_t)t * k, (size_t)k, 1);
 }
 
 cudaError_t launch_topk(const float* zpart, int split, const float* bias, int T, int E, int k, int32_t* idx,

@@ -42,7 +42,7 @@ def test_wait_limit_runs_out_and_the_handle_recovers(name, kw):
     dl = qmoe.DeviceLayer(L)
     try:
         qmoe.qmoe_check_error(dl.handle)                 # clean start
-        qmoe.qmoe_set_wait_limit(dl.handle, 2000)        # far below any tile's wait
+        qmoe.qmoe_set_wait_limit(dl.handle, 100)         # far below one DRAM round trip
         _forward(dl, L.T)
         with pytest.raises(qmoe.QmoeError) as ei:
             qmoe.qmoe_check_error(dl.handle)
