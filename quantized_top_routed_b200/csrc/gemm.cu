@@ -33,22 +33,29 @@
 //
 // Persistent CTAs (one per SM) walk the tile list (segment, 128-row weight
 // block, BN-row token block) built on the device by the schedule kernel;
-// one launch handles the experts of one weight format.  Everything a class
-// touches is private to it: raw producer c, dequantisation group c, issuer
-// c, partial c, and its own raw ring, A ring (TMEM) and B ring (shared
-// memory).  So every ring slot has one producer and one consumer that both
-// walk its uses in order, and a parity wait can never be two phases behind.
+// one launch handles the experts of one weight format.  Each class has its
+// own dequantisation group, issuer, partial (or D slots) and its own raw
+// ring, A ring (TMEM) and B ring (shared memory), and each ring slot has a
+// single producer warp.  So every ring slot has one producer and one
+// consumer that both walk its uses in order, and a parity wait can never be
+// two phases behind.
 //
 // Copy requests.  A TMA request holds the warp that issues it for several
 // hundred cycles whatever its size (up to ~16 KB), while requests from
-// different warps proceed in parallel.  So each class has its own producer
-// warp, requests are large (the weight repack stores each class's stages of
-// a block contiguously and one bulk copy brings NST of them; each K stage of
-// B is one 3-D tensor box of 64 columns x BN rows x 2 column chunks), and the
-// issuer warps issue nothing but MMAs.
+// different warps proceed in parallel.  So copies come from two producer
+// warps, requests are large (the weight repack stores each class's stages
+// of a block contiguously and one bulk copy brings NST of them; each K stage
+// of B is one 3-D tensor box of 64 columns x BN rows x 2 column chunks), and
+// the issuer warps issue nothing but MMAs.
+//
+// Per-stage scaling (INT4 group 128, BN <= 32).  A 128-K stage is one
+// quantisation group, so A holds the exact codes q, each stage's MMAs write
+// a D slot of their own, and the epilogue adds s(row, stage) * D into fp32
+// registers in K order: the group scale is never rounded to bf16.
 // Warp roles, all synchronised through mbarriers:
-//   warps 0, 1   : producer of class 0 / 1 (lane 0): raw weight chunks (bulk
-//                  copies) and B stages (TMA); warp 0 also allocates TMEM
+//   warps 0, 1   : producers (lane 0): raw weight chunks (bulk copies) and B
+//                  stages (TMA) of class 0 / 1, or (BN >= 64) all raw
+//                  chunks / all B stages; warp 0 also allocates TMEM
 //   warps 2, 3   : MMA issuer of class 0 / 1 (warp-uniform loops, one
 //                  elected lane issues)
 //   warps 4..11  : dequantise A into TMEM, group c = warps 4 + 4c .. 7 + 4c;
@@ -98,6 +105,11 @@ struct Cfg {
   static constexpr int SH0 = ((int)kTmemCols - ACC) / 64 / kCls;
   static constexpr int SH = SH0 > 3 ? 3 : SH0;                       // A slots (TMEM) per class
   static constexpr int SA = kCls * SH;
+  // Producers: with wide token blocks (tensor-bound calls) one warp issues
+  // the raw copies of both classes and the other the B boxes, so neither
+  // kind of copy waits behind the other; with narrow ones each class has
+  // its own producer warp issuing both.
+  static constexpr bool SPLIT_PROD = BN >= 64;
   // Scale ring of the per-stage mode: slot i % SC of class c holds the fp32
   // scales of class item i.  SC >= SH + DR: the dequantisation of item
   // i + SC waits for the MMAs of item i + SC - SH, which waited for the D
@@ -139,7 +151,7 @@ struct Tile {
 };
 
 __device__ __forceinline__ Tile decode_tile(int tile, const int32_t* tab_off, const int32_t* seg_off,
-                                            const int32_t* seg_cnt, int n_seg, int bn) {
+                                            const int32_t* seg_cnt, int n_seg, int bn, int group) {
   int lo = 0, hi = n_seg;  // largest seg with tab_off[seg] <= tile
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -148,7 +160,20 @@ __device__ __forceinline__ Tile decode_tile(int tile, const int32_t* tab_off, co
   const int cnt = seg_cnt[lo];
   const int nblk = (cnt + bn - 1) / bn;
   const int local = tile - tab_off[lo];
-  const int mb = local / nblk, nb = local - mb * nblk;
+  int mb, nb;
+  if (group > 0 && nblk > group) {
+    // groups of `group` token blocks; inside a group, weight block major
+    const int nmb = (tab_off[lo + 1] - tab_off[lo]) / nblk;
+    const int per = nmb * group;
+    const int g = local / per;
+    const int gsz = min(group, nblk - g * group);
+    const int rem = local - g * per;
+    mb = rem / gsz;
+    nb = g * group + rem % gsz;
+  } else {
+    mb = local / nblk;
+    nb = local - mb * nblk;
+  }
   Tile t;
   t.seg = lo;
   t.mb = mb;
@@ -371,13 +396,73 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int total = tab_off[n_seg];
   // This CTA's tiles: blockIdx.x + q * gridDim.x for q < nt.
   const int nt = (int)blockIdx.x < total ? (total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+  // Down GEMM: the token blocks of an expert are visited in groups of 8, and
+  // inside a group weight block major, so a group's H rows stay in L2 while
+  // all weight blocks pass over them.  (Gate/up keeps weight block major over
+  // all token blocks: its x rows are small next to W13.)
+  constexpr int kGroup = MAT == 1 ? 8 : 0;
   auto tile_of = [&](int q) { return decode_tile((int)blockIdx.x + q * (int)gridDim.x, tab_off, s_seg_off,
-                                                 s_seg_cnt, n_seg, BN); };
+                                                 s_seg_cnt, n_seg, BN, kGroup); };
 
   if (warp < kMmaWarp0) {
     // ---------------- producer of class c: raw chunks and B stages ----------------
     // Items in order: the raw chunk when an item starts one (NST class stages
     // per bulk copy), then the item's B stage (one 3-D tensor box).
+    if constexpr (C::SPLIT_PROD) {
+    // warp 0: raw chunks of both classes; warp 1: B stages of both classes
+    bool ok = true;
+    uint32_t issued[kCls] = {0, 0};
+    if (warp == kProdWarp0) {
+      for (int q = 0; q < nt && ok; ++q) {
+        const Tile t = tile_of(q);
+        const uint8_t* base = a.experts[t.seg].w[MAT] + (size_t)t.mb * KS * F::SB;
+        for (int m = 0; m < nchunk(0) && ok; ++m) {
+          for (int c = 0; c < kCls; ++c) {
+            const int nc = ncls(c), nch = nchunk(c);
+            if (m >= nch) continue;
+            const uint32_t g = (uint32_t)(q * nch + m);
+            const uint32_t r = c * RH + g % RH, ph = (g / RH) & 1;
+            if (!(ok = warp_wait_backoff(&raw_empty[r], ph ^ 1, abort_flag, kSleepRaw, lim))) break;
+            const uint32_t bytes = (uint32_t)(min(NST, nc - m * NST) * F::SB);
+            const size_t pos = (size_t)(c ? ncls(0) : 0) + (size_t)m * NST;
+            if (lane == 0) {
+              mbar_arrive_expect_tx(&raw_full[r], bytes);
+              bulk_g2s(sRaw + r * C::CHUNK, base + pos * F::SB, bytes, &raw_full[r]);
+            }
+            __syncwarp();
+            issued[c] = g + 1;
+          }
+        }
+      }
+      if (lane == 0)
+        for (int c = 0; c < kCls; ++c) {
+          const uint32_t first = issued[c] > (uint32_t)RH ? issued[c] - RH : 0;
+          for (uint32_t g = first; g < issued[c]; ++g) mbar_wait_drain(&raw_full[c * RH + g % RH], (g / RH) & 1);
+        }
+    } else {
+      for (int q = 0; q < nt && ok; ++q) {
+        const Tile t = tile_of(q);
+        for (int ks = 0; ks < KS; ++ks) {
+          const int c = ks & 1, j = ks >> 1;
+          const uint32_t i = (uint32_t)(q * ncls(c) + j);
+          const uint32_t sb = c * SHB + i % SHB, pb = (i / SHB) & 1;
+          if (!(ok = warp_wait_backoff(&bempty[sb], pb ^ 1, abort_flag, kSleepB, lim))) break;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&bfull[sb], (uint32_t)C::B_STAGE);
+            tma_tile3d(smem_u32(sB + sb * C::B_STAGE), &act_map, 0, t.row0, 2 * ks, &bfull[sb]);
+          }
+          __syncwarp();
+          issued[c] = i + 1;
+        }
+      }
+      if (lane == 0)
+        for (int c = 0; c < kCls; ++c) {
+          const uint32_t first = issued[c] > (uint32_t)SHB ? issued[c] - SHB : 0;
+          for (uint32_t i = first; i < issued[c]; ++i) mbar_wait_drain(&bfull[c * SHB + i % SHB], (i / SHB) & 1);
+        }
+    }
+    __syncwarp();
+    } else {
     const int c = warp - kProdWarp0;
     const int nc = ncls(c), nch = nchunk(c);
     const int first_pos = c ? ncls(0) : 0;   // position of the class's first stage in a block
@@ -420,6 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (uint32_t i = firstb; i < b_issued; ++i) mbar_wait_drain(&bfull[c * SHB + i % SHB], (i / SHB) & 1);
     }
     __syncwarp();
+    }
   } else if (warp < kDQWarp0) {
     // ---------------- MMA issuer of class c ----------------
     // Class stages ks = c, c + 2, ... of every tile, accumulated into partial
