@@ -218,19 +218,33 @@ def make_expert(d: int, I: int, fmt: int, e: int, seed: int = 0) -> Expert:
     return Expert(fmt=fmt, w13=q13, s13=s13, w2=q2, s2=s2)
 
 
-def make_layer(name: str, T: Optional[int] = None, seed: int = 0, **overrides) -> LayerInputs:
-    """Build the named workload (``CONFIGS``) with optional shape overrides."""
+def _config(name: str, T: Optional[int], overrides: dict) -> dict:
     cfg = dict(CONFIGS[name]) if name in CONFIGS else {}
     cfg.update(overrides)
     if T is not None:
         cfg["T"] = T
-    T_, d, E, k, I, S = (cfg[key] for key in ("T", "d", "E", "k", "I", "S"))
+    return cfg
+
+
+def make_router_inputs(name: str, T: Optional[int] = None, seed: int = 0, **overrides):
+    """The named workload's x (bf16 bits), router weights and bias, without
+    the experts: the same arrays make_layer returns for them."""
+    cfg = _config(name, T, overrides)
+    T_, d, E = cfg["T"], cfg["d"], cfg["E"]
     _, r_ss, _, _ = _streams(seed)
     rng = np.random.Generator(np.random.PCG64(r_ss))
     router_w = (rng.standard_normal((E, d), dtype=np.float32) * np.float32(1.0 / np.sqrt(d))).astype(np.float32)
     router_b = zipf_bias(E, cfg["zipf"], seed) if cfg.get("zipf") else None
+    return make_x(T_, d, seed), router_w, router_b
+
+
+def make_layer(name: str, T: Optional[int] = None, seed: int = 0, **overrides) -> LayerInputs:
+    """Build the named workload (``CONFIGS``) with optional shape overrides."""
+    cfg = _config(name, T, overrides)
+    T_, d, E, k, I, S = (cfg[key] for key in ("T", "d", "E", "k", "I", "S"))
+    x, router_w, router_b = make_router_inputs(name, T, seed, **overrides)
     experts = [make_expert(d, I, expert_format(cfg, e), e, seed) for e in range(E + S)]
-    return LayerInputs(name=name, T=T_, d=d, E=E, k=k, I=I, S=S, x=make_x(T_, d, seed),
+    return LayerInputs(name=name, T=T_, d=d, E=E, k=k, I=I, S=S, x=x,
                        router_w=router_w, router_b=router_b, experts=experts, seed=seed)
 
 

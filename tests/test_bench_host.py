@@ -80,3 +80,30 @@ def test_load_report_recovers_a_zipf_exponent():
     assert rep["touched_experts"] == 64 and sum(rep["counts"]) == counts.sum()
     flat = bench.load_report(types.SimpleNamespace(name="decode"), np.full(8, 5))
     assert "zipf_s_fit" not in flat and flat["max_over_mean"] == 1.0
+
+
+@pytest.mark.parametrize("name", ["fine", "mixed"])
+def test_realised_zipf_load_of_the_skewed_workloads(name):
+    """Realised per-expert load of the Zipf-biased workloads, routed by the fp64
+    oracle on the seeded inputs ("OmniMoE" explainer, section 2.2: tasks grouped
+    by expert).  The bias ranks the experts by the Zipf share, so the load must
+    follow that ranking; top-k on the biased logits concentrates it beyond the
+    nominal exponent.  The histogram and the fit printed here are what the
+    bench reports under "load" for the same inputs."""
+    import numpy as np
+    import oracle.qmoe_oracle as O
+    cfg = synth.CONFIGS[name]
+    x, wr, b = synth.make_router_inputs(name)
+    idx = O.topk(O.router_logits(x, wr, b), cfg["k"])
+    counts = np.bincount(idx.ravel(), minlength=cfg["E"])
+    rep = bench.load_report(types.SimpleNamespace(name=name), counts)
+    order = np.argsort(-counts, kind="stable")
+    print(f"{name}: fitted Zipf exponent {rep['zipf_s_fit']} (nominal {cfg['zipf']}), "
+          f"max/mean {rep['max_over_mean']}, touched {rep['touched_experts']}/{cfg['E']}; "
+          f"rows per expert, largest first: {counts[order].tolist()}")
+    assert counts.sum() == cfg["T"] * cfg["k"]
+    assert rep["zipf_s_fit"] > cfg["zipf"]
+    # rank correlation of bias and load (Spearman, no ties in the bias)
+    rb = np.argsort(np.argsort(-b)).astype(np.float64)
+    rc = np.argsort(np.argsort(-counts, kind="stable")).astype(np.float64)
+    assert np.corrcoef(rb, rc)[0, 1] > 0.9
