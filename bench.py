@@ -483,7 +483,7 @@ def cpu_baseline(L, O, args):
             O.forward(L, tokens=oracle_sample_tokens(L, 1, n))
             n += 1
             dt = time.perf_counter() - t0
-    return {"value": round(n / dt, 4), "unit": UNIT, "cores": 1, "host_cores": host_cores(),
+    return {"value": round(n / dt, 4), "unit": UNIT, "cores": 1, "host_cores": host_cores(), "nproc": os.cpu_count(),
             "omp_num_threads": os.environ.get("OMP_NUM_THREADS"), "kind": "oracle",
             "sample": f"{n} tokens of the same batch, one oracle call each (routing, dequantisation of the "
                       f"token's experts, the expert FFNs and the combine in float64), one thread, {dt:.1f} s"}
