@@ -65,7 +65,8 @@ typedef enum {
   QMOE_ERR_UNSUPPORTED = 2,  /* valid but not supported here (e.g. no sm_100 device) */
   QMOE_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
   QMOE_ERR_OOM = 4,          /* device allocation failed in qmoe_create */
-  QMOE_ERR_TIMEOUT = 5       /* a kernel's bounded wait ran out (see qmoe_check_error) */
+  QMOE_ERR_TIMEOUT = 5,      /* a kernel's bounded wait ran out (see qmoe_check_error) */
+  QMOE_ERR_BOUNDS = 6        /* QMOE_DEBUG build only: a device-side bounds check failed */
 } qmoe_status;
 
 /* Expert weight formats ("Quantized Mixture of Experts (Q-MoE)", section 3,
@@ -138,9 +139,18 @@ qmoe_status qmoe_forward_host(qmoe_handle* h, const uint16_t* x_host, int32_t T,
                               void* stream);
 
 /* Synchronise `stream` and report whether any kernel of this handle hit its
- * bounded-wait limit since the last check (QMOE_ERR_TIMEOUT), then clear
- * the flag.  Returns QMOE_OK otherwise. */
+ * bounded-wait limit since the last check (QMOE_ERR_TIMEOUT) or, in the
+ * QMOE_DEBUG build, failed a device-side bounds check (QMOE_ERR_BOUNDS,
+ * reported first), then clear the flags.  Returns QMOE_OK otherwise. */
 qmoe_status qmoe_check_error(qmoe_handle* h, void* stream);
+
+/* 1 in the QMOE_DEBUG build of the library, else 0.  That build (a
+ * stand-in for a device memory checker) checks every index the kernels take
+ * from data (expert ids, token rows, schedule positions, output rows) before
+ * it is used: a failed check skips the access and raises QMOE_ERR_BOUNDS in
+ * the handle's error word instead of faulting.  Results are otherwise the
+ * same bits as the normal build's.  The method has no counterpart to this. */
+int32_t qmoe_debug_build(void);
 
 /* Bound, in SM clock cycles, of every barrier wait inside the grouped GEMM
  * kernels of this handle (0 restores the default of 2^31, about a second).

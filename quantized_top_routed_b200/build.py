@@ -2,9 +2,14 @@
 
 ``python -m quantized_top_routed_b200.build [--force] [--verbose]``
 
-Objects go to ``_build/`` at the repository root; the shared library is
+Objects go to ``_build/`` at the repository root; the shared libraries are
 written next to this file.  The CUDA runtime is linked statically, so the
 library only needs the NVIDIA driver at run time.
+
+Two libraries are built from the same sources: ``libqmoe.so`` and
+``libqmoe_debug.so`` (``-DQMOE_DEBUG``: device-side bounds checks that raise
+QMOE_ERR_BOUNDS instead of faulting).  The binding loads the second only
+when the environment sets ``QMOE_DEBUG=1``.
 """
 from __future__ import annotations
 
@@ -21,6 +26,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libqmoe.so")
+LIB_DEBUG = os.path.join(PKG, "libqmoe_debug.so")
 SOURCES = ["api.cu", "router.cu", "schedule.cu", "gemm.cu", "combine.cu", "repack.cu"]
 HEADERS = ["qmoe_internal.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -45,28 +51,33 @@ def _inputs():
 HASH = LIB + ".srchash"
 
 
-def source_hash() -> str:
+def _flags(debug: bool):
+    return FLAGS + (["-DQMOE_DEBUG"] if debug else [])
+
+
+def source_hash(debug: bool = False) -> str:
     h = hashlib.sha256()
     for p in _inputs():
         with open(p, "rb") as f:
             h.update(os.path.basename(p).encode())
             h.update(f.read())
-    h.update(" ".join(ARCH + FLAGS).encode())
+    h.update(" ".join(ARCH + _flags(debug)).encode())
     return h.hexdigest()
 
 
-def up_to_date() -> bool:
+def up_to_date(debug: bool = False) -> bool:
     """The library exists and was built from exactly the current sources
     (content hash, so copies of the tree with fresh timestamps still match)."""
-    if not (os.path.exists(LIB) and os.path.exists(HASH)):
+    lib = LIB_DEBUG if debug else LIB
+    if not (os.path.exists(lib) and os.path.exists(lib + ".srchash")):
         return False
-    with open(HASH) as f:
-        return f.read().strip() == source_hash()
+    with open(lib + ".srchash") as f:
+        return f.read().strip() == source_hash(debug)
 
 
-def _compile(src: str, verbose: bool) -> str:
-    obj = os.path.join(BUILD, os.path.splitext(src)[0] + ".o")
-    cmd = [nvcc(), *ARCH, *FLAGS, "-c", os.path.join(CSRC, src), "-o", obj]
+def _compile(src: str, verbose: bool, debug: bool = False) -> str:
+    obj = os.path.join(BUILD, "debug" if debug else "", os.path.splitext(src)[0] + ".o")
+    cmd = [nvcc(), *ARCH, *_flags(debug), "-c", os.path.join(CSRC, src), "-o", obj]
     if verbose:
         cmd += ["-Xptxas", "-v"]
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -77,26 +88,37 @@ def _compile(src: str, verbose: bool) -> str:
     return obj
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    lib = LIB_DEBUG if debug else LIB
+    if not force and up_to_date(debug):
+        return lib
+    os.makedirs(os.path.join(BUILD, "debug" if debug else ""), exist_ok=True)
     with concurrent.futures.ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose), SOURCES))
-    tmp = LIB + ".tmp"
+        objs = list(ex.map(lambda s: _compile(s, verbose, debug), SOURCES))
+    tmp = lib + ".tmp"
     cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    with open(HASH, "w") as f:
-        f.write(source_hash())
-    return LIB
+    os.replace(tmp, lib)
+    with open(lib + ".srchash", "w") as f:
+        f.write(source_hash(debug))
+    return lib
+
+
+def build_all(force: bool = False, verbose: bool = False) -> list:
+    """Both libraries: the product one and the QMOE_DEBUG one."""
+    return [build(force, verbose, debug=False), build(force, verbose, debug=True)]
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true", help="print ptxas register/smem usage")
+    ap.add_argument("--debug-only", action="store_true", help="build only libqmoe_debug.so")
+    ap.add_argument("--product-only", action="store_true", help="build only libqmoe.so")
     args = ap.parse_args()
-    print(build(force=args.force, verbose=args.verbose))
+    if not args.product_only:
+        print(build(force=args.force, verbose=args.verbose, debug=True))
+    if not args.debug_only:
+        print(build(force=args.force, verbose=args.verbose))

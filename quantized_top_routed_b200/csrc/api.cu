@@ -211,7 +211,7 @@ qmoe_status route_impl(qmoe_handle* h, const uint16_t* x, const float* logits, i
     StageTimer tm(h, s, QMOE_STAGE_SCHEDULE);
     QMOE_CUDA(launch_schedule(kUsePdl, idx, T, c.k, c.E, tables ? c.n_shared : 0, bn, 2 * c.I / kTileM, c.d / kTileM,
                               h->seg_fmt, counts, offsets, sorted_token, inv_pos, tables ? h->seg_off : nullptr,
-                              tables ? h->seg_cnt : nullptr, h->tiles, h->sched_scratch, s),
+                              tables ? h->seg_cnt : nullptr, h->tiles, h->sched_scratch, h->err, s),
               "schedule launch");
   }
   return QMOE_OK;
@@ -395,7 +395,8 @@ qmoe_status qmoe_forward(qmoe_handle* h, const uint16_t* x, int32_t T, uint16_t*
   {
     // x rows in schedule order (the permutation half of stage 2)
     StageTimer tm(h, s, QMOE_STAGE_SCHEDULE);
-    QMOE_CUDA(launch_permute_rows(kUsePdl, x, h->sorted_token, T * (c.k + c.n_shared), c.d, h->Xp, h->mma_f16, s),
+    QMOE_CUDA(launch_permute_rows(kUsePdl, x, h->sorted_token, T * (c.k + c.n_shared), c.d, h->Xp, h->mma_f16, T,
+                                  h->err, s),
               "permute launch");
   }
   GemmArgs g{};
@@ -404,6 +405,7 @@ qmoe_status qmoe_forward(qmoe_handle* h, const uint16_t* x, int32_t T, uint16_t*
   g.seg_cnt = h->seg_cnt;
   g.n_seg = c.E + c.n_shared;
   g.err = h->err;
+  g.rows = T * (c.k + c.n_shared);
   g.wait_limit = h->wait_limit;
   for (int mat = 0; mat < 2; ++mat) {
     StageTimer tm(h, s, mat == 0 ? QMOE_STAGE_GATE_UP : QMOE_STAGE_DOWN);
@@ -425,7 +427,8 @@ qmoe_status qmoe_forward(qmoe_handle* h, const uint16_t* x, int32_t T, uint16_t*
   }
   {
     StageTimer tm(h, s, QMOE_STAGE_COMBINE);
-    QMOE_CUDA(launch_combine(kUsePdl, h->Y, h->gates, h->inv_pos, T, c.k, c.n_shared, c.d, out, s), "combine launch");
+    QMOE_CUDA(launch_combine(kUsePdl, h->Y, h->gates, h->inv_pos, T, c.k, c.n_shared, c.d, out, h->err, s),
+              "combine launch");
   }
   if (h->profiling) h->profiled_calls++;
   return QMOE_OK;
@@ -454,9 +457,18 @@ qmoe_status qmoe_check_error(qmoe_handle* h, void* stream) {
   if (flag) {
     QMOE_CUDA(cudaMemsetAsync(h->err, 0, sizeof(int), s), "clear error word");
     QMOE_CUDA(cudaStreamSynchronize(s), "stream synchronize");
+    if (flag & kErrBounds) return fail(QMOE_ERR_BOUNDS, "a device-side bounds check failed (QMOE_DEBUG build)");
     return fail(QMOE_ERR_TIMEOUT, "a grouped GEMM kernel hit its bounded-wait limit and aborted");
   }
   return QMOE_OK;
+}
+
+int32_t qmoe_debug_build(void) {
+#ifdef QMOE_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
 }
 
 qmoe_status qmoe_set_wait_limit(qmoe_handle* h, int64_t cycles) {

@@ -34,7 +34,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // before any accumulation, so a token costs one memory round trip.
 __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ Y, const float* __restrict__ gate,
                                                       const int32_t* __restrict__ inv_pos, int T, int k, int S,
-                                                      int d, uint16_t* __restrict__ out) {
+                                                      int d, uint16_t* __restrict__ out, int* __restrict__ err) {
   pdl_wait();                                   // Y is complete past this point
   const int nvec = d >> 3;
   const long long gv = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -47,7 +47,11 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
     if (j < k) {
       const int pos = __ldg(inv_pos + (size_t)t * k + j);
       g[j] = __ldg(gate + (size_t)t * k + j);
-      y[j] = __ldg(reinterpret_cast<const uint4*>(Y + (size_t)pos * d) + v);
+      if (dbg_in_bounds(pos >= 0 && pos < T * k, err)) {
+        y[j] = __ldg(reinterpret_cast<const uint4*>(Y + (size_t)pos * d) + v);
+      } else {
+        y[j] = make_uint4(0u, 0u, 0u, 0u);
+      }
     }
   }
 #pragma unroll
@@ -72,13 +76,15 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
 // 16-byte vector, so each row is read and written with coalesced accesses.
 __global__ void __launch_bounds__(256) permute_rows_kernel(const uint16_t* __restrict__ x,
                                                            const int32_t* __restrict__ sorted_token, int P, int d,
-                                                           uint16_t* __restrict__ xp, int to_f16) {
+                                                           uint16_t* __restrict__ xp, int to_f16, int T,
+                                                           int* __restrict__ err) {
   pdl_wait();                                   // the schedule's permutation is complete past this point
   const int nvec = d >> 3;
   const long long gv = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (gv >= (long long)P * nvec) return;
   const int p = (int)(gv / nvec), v = (int)(gv - (long long)p * nvec);
   const int t = __ldg(sorted_token + p);
+  if (!dbg_in_bounds(t >= 0 && t < T, err)) return;
   uint4 q = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d) + v);
   if (to_f16) {                                 // bf16 -> fp16 (exact inside the fp16 range)
     uint32_t* w = reinterpret_cast<uint32_t*>(&q);
@@ -94,17 +100,17 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const uint16_t* __res
 }  // namespace
 
 cudaError_t launch_permute_rows(bool pdl, const uint16_t* x, const int32_t* sorted_token, int P, int d, uint16_t* xp,
-                                bool to_f16, cudaStream_t s) {
+                                bool to_f16, int T, int* err, cudaStream_t s) {
   const long long n = (long long)P * (d >> 3);
   return launch_ex(permute_rows_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, pdl, x, sorted_token, P,
-                   d, xp, to_f16 ? 1 : 0);
+                   d, xp, to_f16 ? 1 : 0, T, err);
 }
 
 cudaError_t launch_combine(bool pdl, const uint16_t* Y, const float* gate, const int32_t* inv_pos, int T, int k, int S, int d,
-                           uint16_t* out, cudaStream_t s) {
+                           uint16_t* out, int* err, cudaStream_t s) {
   const long long n = (long long)T * (d >> 3);
   return launch_ex(combine_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, pdl, Y, gate, inv_pos, T, k, S,
-                   d, out);
+                   d, out, err);
 }
 
 }  // namespace qmoe

@@ -393,7 +393,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = tab_off[n_seg];
+#ifdef QMOE_DEBUG
+  // The tile tables come from data (the schedule's output): check them
+  // before any role uses them, and give every role of the CTA no tiles if
+  // they are bad, so all roles stay consistent.
+  volatile int* tab_bad = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
+  if (tid == 0) {
+    int bad = tab_off[0] != 0;
+    for (int i = 0; i < n_seg && !bad; ++i) {
+      const int cnt = s_seg_cnt[i], tiles = tab_off[i + 1] - tab_off[i];
+      const int want = ((cnt + BN - 1) / BN) * a.MB;
+      bad = cnt < 0 || s_seg_off[i] < 0 || s_seg_off[i] + cnt > a.rows || (tiles != 0 && tiles != want);
+    }
+    *tab_bad = bad;
+  }
+  __syncthreads();
+  const bool tab_ok = dbg_in_bounds(*tab_bad == 0, tid == 0 ? a.err : nullptr);
+#else
+  constexpr bool tab_ok = true;
+#endif
+  const int total = tab_ok ? tab_off[n_seg] : 0;
   // This CTA's tiles: blockIdx.x + q * gridDim.x for q < nt.
   const int nt = (int)blockIdx.x < total ? (total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
   // Down GEMM: the token blocks of an expert are visited in groups of 8, and

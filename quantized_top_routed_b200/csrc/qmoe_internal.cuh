@@ -18,6 +18,19 @@ constexpr int kTileM = 128;       // weight rows per GEMM tile (MMA M)
 
 // Error bits written to the handle's device error word.
 constexpr int kErrTimeout = 1;
+constexpr int kErrBounds = 2;
+
+// Bounds check of the QMOE_DEBUG build: when `ok` is false the handle's
+// error word gets kErrBounds and the caller skips the access.  In the normal
+// build the check is the constant true and costs nothing.
+#ifdef QMOE_DEBUG
+__device__ __forceinline__ bool dbg_in_bounds(bool ok, int* err) {
+  if (!ok && err) atomicOr(err, kErrBounds);
+  return ok;
+}
+#else
+__device__ __forceinline__ bool dbg_in_bounds(bool, int*) { return true; }
+#endif
 
 // One expert's weights after repacking (device pointers, owned by the handle).
 // mat 0 = gate/up (W13, K = d), mat 1 = down (W2, K = I).
@@ -60,6 +73,7 @@ struct GemmArgs {
   int MB;                     // 128-row weight blocks per expert matrix
   uint16_t* out;              // H [P][I] or Y [P][d]
   int out_ld;
+  int rows;                   // rows of act and out (T * (k + shared))
   int* err;                   // device error word
   long long wait_limit;       // SM cycles a bounded wait may last before the kernel aborts
 };
@@ -372,7 +386,7 @@ __host__ __device__ inline int tile_table_offset(int mat, int fmt, int n_seg) {
 cudaError_t launch_schedule(bool pdl, const int32_t* idx, int T, int k, int E, int S, int bn, int mb3, int mb4,
                             const int32_t* seg_fmt, int32_t* counts, int32_t* offsets, int32_t* sorted_token,
                             int32_t* inv_pos, int32_t* seg_off, int32_t* seg_cnt, int32_t* tiles, int32_t* scratch,
-                            cudaStream_t s);
+                            int* err, cudaStream_t s);
 size_t schedule_scratch_ints(int max_tokens, int E);
 
 bool gemm_bn_supported(int bn);
@@ -383,10 +397,10 @@ cudaError_t launch_grouped_gemm(bool pdl, const GemmArgs& a, const CUtensorMap& 
 // xp[p] = x[sorted_token[p]] for p < P (activation rows in schedule order).
 // to_f16: write the rows as fp16 (the fp16 MMA mode) instead of copying bf16.
 cudaError_t launch_permute_rows(bool pdl, const uint16_t* x, const int32_t* sorted_token, int P, int d, uint16_t* xp,
-                                bool to_f16, cudaStream_t s);
+                                bool to_f16, int T, int* err, cudaStream_t s);
 
 cudaError_t launch_combine(bool pdl, const uint16_t* Y, const float* gate, const int32_t* inv_pos, int T, int k, int S,
-                           int d, uint16_t* out, cudaStream_t s);
+                           int d, uint16_t* out, int* err, cudaStream_t s);
 
 cudaError_t launch_repack(int fmt, int mat, const void* w, const void* scale, int rows, int K, int I,
                           uint8_t* dst, float* dst_spc, cudaStream_t s);

@@ -33,7 +33,9 @@ static_assert(kSmemPipe >= RT * kMaxE * 4, "the top-k tail keeps the tile's logi
 
 // One warp: softmax + top-k + renormalisation of the E logits of NT tokens
 // at once (the tokens' shuffle chains interleave; each token's arithmetic is
-// the same as with NT = 1).  logit(u, e) gives the fp32 logit of expert e
+// the same as with NT = 1).  NaN logits are taken as -inf, so every pick is
+// an expert index in [0, E) whatever the input (ties, -inf included, go to
+// the lower index).  logit(u, e) gives the fp32 logit of expert e
 // (bias included) for the warp's token u; token u's outputs go to
 // idx0 + u * ld and gate0 + u * ld when u < nvalid.
 template <int EPL, int NT, class LogitFn>
@@ -51,7 +53,8 @@ __device__ __forceinline__ void topk_tokens(LogitFn logit, int E, int k, int lan
       const int e = lane + 32 * i;
       const bool ok = e < E;
       if (ok) live |= 1u << (u * EPL + i);
-      z[u][i] = ok ? logit(u, e) : -INFINITY;
+      const float v = ok ? logit(u, e) : -INFINITY;
+      z[u][i] = v == v ? v : -INFINITY;   // a NaN logit ranks below every number, so the picks stay valid experts
       m[u] = fmaxf(m[u], z[u][i]);
     }
   }

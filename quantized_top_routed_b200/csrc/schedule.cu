@@ -37,7 +37,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int32_t* __restrict__ seg_fmt, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                     int32_t* __restrict__ sorted_token, int32_t* __restrict__ inv_pos,
                     int32_t* __restrict__ seg_off, int32_t* __restrict__ seg_cnt, int32_t* __restrict__ tiles,
-                    int32_t* __restrict__ hist_global, int hist_in_smem) {
+                    int32_t* __restrict__ hist_global, int hist_in_smem, int* __restrict__ err) {
   extern __shared__ int32_t hist_smem[];
   __shared__ uint32_t bal[32][kMaxE];
   __shared__ int32_t s_cnt[kMaxE + kMaxShared];
@@ -55,7 +55,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool valid = t < T;
     int my[kMaxK];
 #pragma unroll
-    for (int j = 0; j < kMaxK; ++j) my[j] = (valid && j < k) ? idx[(size_t)t * k + j] : -1;
+    for (int j = 0; j < kMaxK; ++j) {
+      my[j] = (valid && j < k) ? idx[(size_t)t * k + j] : -1;
+      if (valid && j < k && !dbg_in_bounds(my[j] >= 0 && my[j] < E, err)) my[j] = -1;
+    }
     for (int w0 = 0; w0 < E; w0 += 32) {
       uint32_t m = 0;
 #pragma unroll
@@ -115,7 +118,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int p = tid; p < P; p += kThreads) {
     const int t = p / k;
     const int e = idx[p];
+    if (!dbg_in_bounds(e >= 0 && e < E, err)) continue;
     const int pos = s_off[e] + hist[(t >> 5) * E + e] + inv_pos[p];
+    if (!dbg_in_bounds(pos >= 0 && pos < P, err)) continue;
     sorted_token[pos] = t;
     inv_pos[p] = pos;
   }
@@ -161,7 +166,7 @@ size_t schedule_scratch_ints(int max_tokens, int E) { return (size_t)((max_token
 cudaError_t launch_schedule(bool pdl, const int32_t* idx, int T, int k, int E, int S, int bn, int mb3, int mb4,
                             const int32_t* seg_fmt, int32_t* counts, int32_t* offsets, int32_t* sorted_token,
                             int32_t* inv_pos, int32_t* seg_off, int32_t* seg_cnt, int32_t* tiles, int32_t* scratch,
-                            cudaStream_t s) {
+                            int* err, cudaStream_t s) {
   // chunk histograms live in shared memory when they fit next to the static arrays
   const size_t hist_bytes = (size_t)((T + 31) / 32) * E * sizeof(int32_t);
   const int in_smem = hist_bytes <= kHistSmemMax;
@@ -171,7 +176,7 @@ cudaError_t launch_schedule(bool pdl, const int32_t* idx, int T, int k, int E, i
     if (e != cudaSuccess) return e;
   }
   return launch_ex(schedule_kernel, dim3(1), dim3(kThreads), dyn, s, pdl, idx, T, k, E, S, bn, mb3, mb4, seg_fmt,
-                   counts, offsets, sorted_token, inv_pos, seg_off, seg_cnt, tiles, scratch, in_smem);
+                   counts, offsets, sorted_token, inv_pos, seg_off, seg_cnt, tiles, scratch, in_smem, err);
 }
 
 }  // namespace qmoe

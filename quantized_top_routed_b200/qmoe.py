@@ -23,6 +23,7 @@ QMOE_ERR_UNSUPPORTED = 2
 QMOE_ERR_CUDA = 3
 QMOE_ERR_OOM = 4
 QMOE_ERR_TIMEOUT = 5
+QMOE_ERR_BOUNDS = 6
 
 W_INT8_PC = 1
 W_INT4_G128 = 2
@@ -32,7 +33,7 @@ STAGES = ("router", "schedule", "gate_up", "down", "combine")
 
 EXPORTS = ("qmoe_create", "qmoe_route", "qmoe_forward", "qmoe_forward_host", "qmoe_check_error",
            "qmoe_profile", "qmoe_profile_read", "qmoe_launches_per_forward", "qmoe_destroy",
-           "qmoe_last_error", "qmoe_route_topk_noalloc", "qmoe_set_wait_limit")
+           "qmoe_last_error", "qmoe_route_topk_noalloc", "qmoe_set_wait_limit", "qmoe_debug_build")
 
 
 class QmoeError(RuntimeError):
@@ -54,20 +55,28 @@ class qmoe_expert(ctypes.Structure):
 _lib = None
 
 
+def debug_requested() -> bool:
+    """QMOE_DEBUG=1 in the environment selects the bounds-checking build."""
+    return os.environ.get("QMOE_DEBUG") == "1"
+
+
 def library_path() -> str:
-    return _build.LIB
+    return _build.LIB_DEBUG if debug_requested() else _build.LIB
 
 
 def load(build_if_missing: bool = True) -> ctypes.CDLL:
-    """Load libqmoe.so (building it in-tree first when it is missing or stale)."""
+    """Load libqmoe.so, or libqmoe_debug.so when QMOE_DEBUG=1 (building it
+    in-tree first when it is missing or stale)."""
     global _lib
     if _lib is not None:
         return _lib
-    if build_if_missing and not _build.up_to_date():
-        _build.build()
-    if not os.path.exists(_build.LIB):
-        raise OSError(f"{_build.LIB} is missing; run python -m quantized_top_routed_b200.build")
-    lib = ctypes.CDLL(_build.LIB)
+    debug = debug_requested()
+    path = library_path()
+    if build_if_missing and not (_build.up_to_date(debug=True) if debug else _build.up_to_date()):
+        _build.build(debug=debug)
+    if not os.path.exists(path):
+        raise OSError(f"{path} is missing; run python -m quantized_top_routed_b200.build")
+    lib = ctypes.CDLL(path)
     vp, i32, f32p = ctypes.c_void_p, ctypes.c_int32, ctypes.POINTER(ctypes.c_float)
     lib.qmoe_create.argtypes = [ctypes.POINTER(qmoe_config), vp, vp, ctypes.POINTER(qmoe_expert),
                                 ctypes.POINTER(vp)]
@@ -84,6 +93,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.qmoe_last_error.restype = ctypes.c_char_p
     lib.qmoe_route_topk_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp]
     lib.qmoe_set_wait_limit.argtypes = [vp, ctypes.c_int64]
+    lib.qmoe_debug_build.argtypes = []
+    lib.qmoe_debug_build.restype = i32
     for name in ("qmoe_create", "qmoe_route", "qmoe_forward", "qmoe_forward_host", "qmoe_check_error",
                  "qmoe_profile", "qmoe_profile_read", "qmoe_destroy", "qmoe_route_topk_noalloc",
                  "qmoe_set_wait_limit"):

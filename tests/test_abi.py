@@ -104,3 +104,20 @@ def test_noalloc_route_validates_before_touching_the_device(T, d, E, k, why):
         qmoe.qmoe_route_topk_noalloc(16, 16, None, T, d, E, k, 16, 16)
     assert ei.value.status == qmoe.QMOE_ERR_INVALID
     assert why in str(ei.value)
+
+
+def test_the_product_library_is_not_the_debug_build():
+    assert qmoe.load().qmoe_debug_build() == 0
+
+
+def test_debug_library_builds_and_exports_the_same_symbols():
+    """The QMOE_DEBUG twin (device-side bounds checks that raise
+    QMOE_ERR_BOUNDS instead of faulting) builds from the same sources and has
+    the same C ABI; it reports itself through qmoe_debug_build()."""
+    path = qmoe._build.build(debug=True)
+    assert path == qmoe._build.LIB_DEBUG and qmoe._build.up_to_date(debug=True)
+    lib = ctypes.CDLL(path)
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} missing from the debug build"
+    lib.qmoe_debug_build.restype = ctypes.c_int32
+    assert lib.qmoe_debug_build() == 1
