@@ -35,7 +35,7 @@ def _forward(dl, T):
 
 @pytest.mark.parametrize("name,kw", [
     ("tiny", dict(T=64)),                       # INT8, 128-row token blocks
-    ("decode", dict(T=32, d=512, I=256)),       # INT4, 16-row token blocks, two accumulator sets
+    ("decode", dict(T=32, d=512, I=256)),       # INT4 with per-stage scaling, 16-row token blocks
 ])
 def test_wait_limit_runs_out_and_the_handle_recovers(name, kw):
     L = synth.make_layer(name, **kw)
