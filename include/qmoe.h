@@ -182,9 +182,11 @@ qmoe_status qmoe_destroy(qmoe_handle* h);
 /* Thread-local text of the last failure in this thread ("" if none). */
 const char* qmoe_last_error(void);
 
-/* Stage 1 (router logits, softmax, top-k, renormalised gates) without a
- * handle and without allocating anything.  The method as published has no
- * counterpart to this call: it exists for callers that cannot allocate
+/* Stage 1 (router logits, softmax, top-k, renormalised gates: the gating
+ * network with top-k routing of "Quantized Mixture of Experts (Q-MoE)",
+ * section 3 "Components", with the softmax mixing weights of "FineRMoE",
+ * Sparse Sum Layer) without a handle and without allocating anything.  The
+ * method as published has no counterpart to calling it this way: it exists for callers that cannot allocate
  * device memory at the point where they route, for example a serving loop
  * whose memory is entirely held by another allocator (a caching or arena
  * allocator that owns all of HBM), or one that must not take the device-wide
