@@ -1,8 +1,10 @@
 """Pins for the number-format claims the GPU path relies on (no GPU needed):
 e4m3 codes are exact in fp16 and in bf16, bf16 activations inside the fp16
 normal range are exact in fp16, INT4 codes and INT8 codes are exact in bf16,
-so the only rounding the dequantisation adds is the one stated (INT4:
-bf16(q * s))."""
+so the only rounding the dequantisation adds is the one stated.  INT4 with
+token blocks of up to 32 rows: none, because the codes q are the MMA input
+and the bf16 group scale, exact in fp32, multiplies each 128-K stage's fp32
+partial sum.  INT4 with wider blocks: bf16(q * s)."""
 import numpy as np
 
 import oracle.qmoe_oracle as O
@@ -48,8 +50,20 @@ def test_int4_and_int8_codes_are_exact_in_bf16():
     assert _is_bf16_exact(q4) and _is_bf16_exact(q8)
 
 
+def test_bf16_group_scales_are_exact_in_fp32():
+    # the per-stage scaling converts the stored bf16 scale to fp32 by a shift
+    # of its bits; every bf16 value, subnormals included, is an fp32 value
+    bits = np.arange(0, 0x10000, dtype=np.uint32)
+    bits = bits[((bits >> 7) & 0xFF) != 0xFF]                     # finite values only
+    f32 = _bf16_bits_to_f32(bits)
+    back = (f32.view(np.uint32) >> 16).astype(np.uint32)
+    assert np.array_equal(back, bits)
+    assert np.all(f32.astype(np.float64) == f32)
+
+
 def test_int4_product_rounding_is_within_half_a_bf16_ulp():
-    # bf16(q * s) for bf16 scales s: one RNE rounding to 8 significant bits,
+    # bf16(q * s) for bf16 scales s (token blocks wider than 32 rows): one RNE
+    # rounding to 8 significant bits,
     # relative error <= 2^-8 (the unit roundoff of bf16).  q * s of two bf16
     # values has at most 16 significant bits, so the fp32 step below is exact.
     rng = np.random.default_rng(1)
