@@ -39,7 +39,8 @@ METRIC = "MoE-layer tokens/s on 1xB200; % of HBM / tensor-core roofline"
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
 ROOF_TIMING = ("CUDA events around every gate/up launch on its stream, in a second pass of the same steps "
-               "(L2 flushed between steps); peak = the measured burst figure")
+               "(L2 flushed between steps); avg_launch_ms is the gate/up time per step, summed over its "
+               "launches_per_step launches (one per weight format); peak = the measured burst figure")
 
 
 # ---------------------------------------------------------------------------
@@ -322,14 +323,18 @@ def measure_layer(args, name, T, rank, world, dev, peaks, flush, headline):
     e2e_ms, e2e_value = job_rate(world, T, sum(e2e_times) / len(e2e_times), dev)
 
     # ---- roofline of the dominant kernel -----------------------------------
+    # gate/up time per step: the sum over its launches (one per weight format
+    # present, two in the mixed layer), against the whole gate/up work
     gu_ms = stage_ms["gate_up"] / max(calls, 1)
+    gu_launches = len({e.fmt for e in L.experts})
     if L.name in ("decode", "tiny"):
         algo = gate_up_bytes(L, touched)
         achieved = algo / (gu_ms / 1e3) / 1e9
         roof = {"kernel": "grouped_gemm gate/up (SwiGLU)", "bound": "hbm", "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "traffic": traffic_from_profiles(L, "gate_up"), "peak_source": peaks["source"],
-                "algorithmic_bytes": algo, "avg_launch_ms": round(gu_ms, 5), "timing": ROOF_TIMING}
+                "algorithmic_bytes": algo, "avg_launch_ms": round(gu_ms, 5),
+                "launches_per_step": gu_launches, "timing": ROOF_TIMING}
     else:
         fl = gate_up_flops(L)
         achieved = fl / (gu_ms / 1e3) / 1e12
@@ -338,7 +343,8 @@ def measure_layer(args, name, T, rank, world, dev, peaks, flush, headline):
                 "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                 "frac_of_sustained_peak": round(achieved / peaks["bf16_tflops_sustained"], 4),
                 "traffic": traffic_from_profiles(L, "gate_up"), "peak_source": peaks["source"],
-                "algorithmic_flops": fl, "avg_launch_ms": round(gu_ms, 5), "timing": ROOF_TIMING}
+                "algorithmic_flops": fl, "avg_launch_ms": round(gu_ms, 5),
+                "launches_per_step": gu_launches, "timing": ROOF_TIMING}
 
     rec = {
         "value": round(value, 1), "unit": UNIT, "ms_per_step": round(ms, 5), "steps": steps,
